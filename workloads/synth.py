@@ -1,0 +1,119 @@
+"""Seeded synthetic inputs shared by the oracle tests, the GPU tests and the bench.
+
+This module holds no arithmetic of the method. It draws standard normals from
+numpy's ``Generator(PCG64(seed))`` in float32, in the fixed order
+q, k, v, gate logits, beta logits, initial state, scales and shifts them to the
+workload's distributions, and rounds the bf16 tensors to bf16 with
+round-to-nearest-even.  Both sides of a parity test receive exactly the same
+values: the GPU side the bf16 bit patterns, the oracle the same values widened
+to float32 (exact).
+
+Layouts (row-major, contiguous):
+  q, k      [B, T, H, d_k]
+  v         [B, T, H, d_v]
+  gate      [B, ceil(T / frame_len), H]   one logit per latent frame and head
+  beta      [B, T, H]                     one logit per token and head
+  state     [B, H, d_k, d_v]              float32
+"""
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+from .configs import Workload
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bf16 (ties to even); returns float32."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32)
+    r = (u >> np.uint32(16)) & np.uint32(1)
+    u = u + np.uint32(0x7FFF) + r
+    u &= np.uint32(0xFFFF0000)
+    return u.view(np.float32)
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Upper 16 bits of float32 values that are already bf16-representable."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    return (x.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+@dataclass
+class Inputs:
+    q: np.ndarray
+    k: np.ndarray
+    v: np.ndarray
+    gate: np.ndarray
+    beta: np.ndarray
+    state: Optional[np.ndarray]
+    io_dtype: str
+    frame_len: int
+
+    @property
+    def shape(self):
+        B, T, H, dk = self.q.shape
+        return B, H, T, dk, self.v.shape[3]
+
+
+def _normal(rng, shape, mean=0.0, std=1.0):
+    x = rng.standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        x *= np.float32(std)
+    if mean != 0.0:
+        x += np.float32(mean)
+    return x
+
+
+def draw(rng: np.random.Generator, B: int, H: int, T: int, d_k: int, d_v: int,
+         frame_len: int, io_dtype: str, gate_mean: float, gate_std: float,
+         beta_mean: float = 0.0, beta_std: float = 1.0,
+         state_std: Optional[float] = None) -> Inputs:
+    """Draw one set of inputs from ``rng`` in the fixed order q, k, v, gate, beta, state."""
+    F = -(-T // frame_len)
+    q = _normal(rng, (B, T, H, d_k))
+    k = _normal(rng, (B, T, H, d_k))
+    v = _normal(rng, (B, T, H, d_v))
+    gate = _normal(rng, (B, F, H), gate_mean, gate_std)
+    beta = _normal(rng, (B, T, H), beta_mean, beta_std)
+    state = None
+    if state_std is not None:
+        state = _normal(rng, (B, H, d_k, d_v), 0.0, state_std)
+    if io_dtype == "bf16":
+        q, k, v = bf16_round(q), bf16_round(k), bf16_round(v)
+    elif io_dtype != "f32":
+        raise ValueError(io_dtype)
+    return Inputs(q, k, v, gate, beta, state, io_dtype, frame_len)
+
+
+def make_inputs(w: Workload, T: Optional[int] = None, seed: Optional[int] = None) -> Inputs:
+    """Inputs of one call of workload ``w`` (optionally with another T or seed)."""
+    rng = np.random.Generator(np.random.PCG64(w.seed if seed is None else seed))
+    return draw(rng, w.B, w.H, w.T if T is None else T, w.d_k, w.d_v, w.frame_len,
+                w.io_dtype, w.gate_mean, w.gate_std, w.beta_mean, w.beta_std, w.state_std)
+
+
+def make_session_blocks(w: Workload, n_blocks: Optional[int] = None):
+    """Batched streaming: session s draws from seed ``session_seed_base + s``.
+
+    Per session the generator first draws the initial state [H, d_k, d_v]
+    (N(0, state_std)), then each block's q, k, v, gate, beta in turn.  The
+    sessions are stacked along B.  Returns (initial_state, [Inputs per block]);
+    the per-block Inputs carry ``state=None``.
+    """
+    n_blocks = w.blocks if n_blocks is None else n_blocks
+    base = w.session_seed_base if w.session_seed_base is not None else 1000
+    rngs = [np.random.Generator(np.random.PCG64(base + s)) for s in range(w.B)]
+    std = w.state_std if w.state_std is not None else 0.0
+    state0 = np.stack([_normal(r, (w.H, w.d_k, w.d_v), 0.0, std) for r in rngs])
+    blocks = []
+    for _ in range(n_blocks):
+        parts = [draw(r, 1, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.io_dtype,
+                      w.gate_mean, w.gate_std, w.beta_mean, w.beta_std, None) for r in rngs]
+        blocks.append(Inputs(
+            q=np.concatenate([p.q for p in parts]), k=np.concatenate([p.k for p in parts]),
+            v=np.concatenate([p.v for p in parts]), gate=np.concatenate([p.gate for p in parts]),
+            beta=np.concatenate([p.beta for p in parts]), state=None,
+            io_dtype=w.io_dtype, frame_len=w.frame_len))
+    return state0, blocks
