@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""GDN forward benchmark on B200: tokens/s per layer on the minute-scale SANA-WM layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: B = 1, H = 20, d_k = d_v = 112, T = 106,480 tokens (121 latent frames
+of 880 tokens), chunk 64, bf16 q/k/v/out, float32 logits and state, seeded
+synthetic inputs; one step = 20 layer calls back to back (one buffer set of
+1.9 GB, larger than the 126 MB L2, so no call finds its inputs in L2).
+
+Multi-GPU: one process per GPU (torchrun); the layer's (batch, head) chains are
+independent, so every rank runs the same per-GPU workload with no collective
+on the data path ("weak" scaling); the step time is the max over ranks.
+
+Prints ONE JSON line from rank 0.  ``--impl reference`` times the float64 CPU
+oracle on a bounded sample of the same workload instead (rank 0 only).
+"""
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GDN fwd tokens/s per layer (20 heads x d112) on 1 B200; % of roofline"
+UNIT = "tokens/s"
+BYTES_PER_TOKEN_HEAD = 900          # q, k, v in + out (bf16, d = 112) + beta logit (f32)
+CHUNKED_FLOPS_PER_TOKEN_HEAD = 146944   # 10 C d + 6 d^2 at C = 64, d = 112
+KERNEL_SOURCES = ["hybrid_linear_attention_frame_b200/csrc/gdn_tc.cu",
+                  "hybrid_linear_attention_frame_b200/csrc/gdn_ffma.cu",
+                  "hybrid_linear_attention_frame_b200/csrc/gdn_common.cuh"]
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=None, help="layer calls per step (default 20)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target wall time of the oracle sample")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (rank setup, barrier, max over ranks)
+# ----------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(backend, world, timeout_s=120):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend,
+                                timeout=datetime.timedelta(seconds=timeout_s))
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a float over all ranks (every rank gets the result)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(tokens_per_rank: float, elapsed_s_this_rank: float, world: int, device=None):
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    slowest = max_over_ranks(elapsed_s_this_rank, world, device)
+    return tokens_per_rank * world / slowest, slowest
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples nvidia-smi every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="gdn_clocks_", suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "200", "-f", self.path]
+            if self.uuid:
+                cmd[1:1] = ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 10:
+                        rows.append(parts)
+            os.unlink(self.path)
+        except OSError:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "", 1).isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "", 1).isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# roofline bookkeeping
+# ----------------------------------------------------------------------------
+
+def algorithmic_bytes(w, state_in: bool, state_out: bool) -> int:
+    """Bytes one gdn_forward call must move at least: q, k, v, out (bf16), the
+    beta logits, the per-frame gate logits and the state (float32)."""
+    th = w.B * w.T * w.H
+    b = th * (2 * w.d_k * 2 + w.d_v * 2 + w.d_v * 2 + 4)
+    b += w.B * w.n_frames * w.H * 4
+    st = w.B * w.H * w.d_k * w.d_v * 4
+    return b + (st if state_in else 0) + (st if state_out else 0)
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """dram bytes per launch from the committed ncu summary, if the kernel sources
+    are the ones it was captured from; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None, None
+    if rec.get("kernel_source_sha") != kernel_source_sha():
+        return None, rec.get("kernel")
+    return rec.get("dram_bytes_per_launch"), rec.get("kernel")
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and reference arm)
+# ----------------------------------------------------------------------------
+
+def slice_tokens(inp, n_tok):
+    """The first n_tok tokens of every (batch, head) chain, with their frames' gates."""
+    from workloads import Inputs
+    F = -(-n_tok // inp.frame_len)
+    return Inputs(q=inp.q[:, :n_tok], k=inp.k[:, :n_tok], v=inp.v[:, :n_tok],
+                  gate=inp.gate[:, :F], beta=inp.beta[:, :n_tok], state=None,
+                  io_dtype=inp.io_dtype, frame_len=inp.frame_len)
+
+
+def oracle_sample_size(inp, seconds, threads):
+    """Tokens per chain the oracle processes in about `seconds` (whole frames)."""
+    from oracle import gdn_reference as R
+    fl = inp.frame_len
+    probe = slice_tokens(inp, fl)
+    t0 = time.perf_counter()
+    R.c_forward(probe, None, n_threads=threads, want_state=False)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    frames = max(1, min(inp.q.shape[1] // fl, int(seconds / dt)))
+    return frames * fl
+
+
+def time_oracle(inp, n_tok, threads, repeats=1):
+    from oracle import gdn_reference as R
+    sub = slice_tokens(inp, n_tok)
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        R.c_forward(sub, None, n_threads=threads, want_state=True)
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def oracle_threads(w):
+    return max(1, min(os.cpu_count() or 1, w.B * w.H))
+
+
+def cpu_baseline(w, inp, seconds):
+    threads = oracle_threads(w)
+    n_tok = oracle_sample_size(inp, seconds, threads)
+    (dt,) = time_oracle(inp, n_tok, threads)
+    return {"value": w.B * n_tok / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"float64 C token recurrence, first {n_tok} tokens of all {w.B * w.H} "
+                      f"(batch, head) chains of one layer, {threads} OpenMP threads "
+                      f"(host has {os.cpu_count()} cores), {dt:.2f} s"}
+
+
+def run_reference(args, w, rank, world):
+    """Reference arm: the float64 CPU oracle on bounded samples of the same workload."""
+    if rank != 0:
+        return None
+    from workloads import make_inputs
+    inp = make_inputs(w)
+    threads = oracle_threads(w)
+    budget = 150.0 / max(1, args.steps + args.warmup)      # whole run within a few minutes
+    n_tok = oracle_sample_size(inp, min(args.cpu_seconds, budget), threads)
+    time_oracle(inp, n_tok, threads, repeats=args.warmup)
+    times = time_oracle(inp, n_tok, threads, repeats=args.steps)
+    per_step = sum(times) / len(times)
+    value = w.B * n_tok / per_step
+    sample = (f"float64 C token recurrence, first {n_tok} tokens of all {w.B * w.H} chains "
+              f"of one layer per step, {threads} OpenMP threads (host has {os.cpu_count()} cores)")
+    return {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, args.layers or w.layers),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def workload_config(w, layers):
+    return {"workload": f"{w.name}: minute-scale SANA-WM GDN layer, B={w.B} H={w.H} "
+                        f"T={w.T} d_k=d_v={w.d_k}, frame {w.frame_len} tokens, chunk {w.chunk_len}, "
+                        f"{layers} layers back-to-back per step",
+            "B": w.B, "H": w.H, "T": w.T, "d_k": w.d_k, "d_v": w.d_v, "frame_len": w.frame_len,
+            "chunk_len": w.chunk_len, "layers_per_step": layers,
+            "gate_logits": f"N({w.gate_mean}, {w.gate_std})", "seed": w.seed,
+            "l2": "inputs larger than L2 (1.9 GB per layer vs 126 MB)",
+            "parallelism": "weak: every rank runs the full layer set on its own GPU"}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args, w, rank, world, local):
+    import numpy as np
+    import torch
+    import hybrid_linear_attention_frame_b200 as G
+    from workloads import bf16_bits, make_inputs
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init("nccl", world)
+    layers = args.layers or w.layers
+    G.load()
+
+    inp = make_inputs(w)
+    def bf16(x):
+        return torch.from_numpy(bf16_bits(x).view(np.int16)).view(torch.bfloat16)
+    h_q, h_k, h_v = bf16(inp.q), bf16(inp.k), bf16(inp.v)
+    h_g = torch.from_numpy(inp.gate)
+    h_b = torch.from_numpy(inp.beta)
+    q, k, v, g, b = (x.to(device) for x in (h_q, h_k, h_v, h_g, h_b))
+    out = torch.empty_like(v)
+    st_out = torch.empty((w.B, w.H, w.d_k, w.d_v), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    sptr = stream.cuda_stream
+    lib = G.load()
+    dims = (w.B, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.chunk_len)
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), b.data_ptr(), None,
+            st_out.data_ptr(), out.data_ptr())
+
+    def layer_call():
+        st = lib.gdn_forward(*ptrs, *dims, sptr)
+        if st != 0:
+            raise G.GdnError(st, "gdn_forward")
+
+    for _ in range(args.warmup):
+        for _ in range(layers):
+            layer_call()
+    torch.cuda.synchronize(device)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps * layers)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        uuid = None
+    clocks = ClockSampler(uuid).start() if rank == 0 else None
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    t_start.record(stream)
+    i = 0
+    for _ in range(args.steps):
+        for _ in range(layers):
+            ev[i][0].record(stream)
+            layer_call()
+            ev[i][1].record(stream)
+            i += 1
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    clock_rec = clocks.stop() if clocks else None
+    dev_status = G.gdn_get_last_device_status()
+    if dev_status != G.GDN_OK:
+        raise G.GdnError(dev_status, "device status after the timed region")
+
+    elapsed_s = t_start.elapsed_time(t_end) / 1e3
+    tokens_per_rank = w.B * w.T * layers * args.steps
+    value, slowest = aggregate_throughput(tokens_per_rank, elapsed_s, world, device)
+    ms_per_step = slowest * 1e3 / args.steps
+    launch_ms = [s.elapsed_time(e) for (s, e) in ev]
+    avg_launch_s = statistics.mean(launch_ms) / 1e3
+
+    peaks, peak_kind = measured_peaks()
+    abytes = algorithmic_bytes(w, state_in=False, state_out=True)
+    achieved = abytes / avg_launch_s / 1e9
+    traffic, traffic_kernel = recorded_traffic()
+    path = G.gdn_bf16_path(w.d_k, w.d_v, w.chunk_len)
+    kernel = "gdn_chunk_tc_kernel" if path == 1 else "chunk_ffma_kernel<bf16,64>"
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic if traffic_kernel == kernel else None,
+                "kernel": kernel, "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
+                "algorithmic_bytes_per_launch": abytes,
+                "avg_launch_us": round(avg_launch_s * 1e6, 2),
+                "tensor_flops_frac": round(
+                    CHUNKED_FLOPS_PER_TOKEN_HEAD * w.B * w.T * w.H / avg_launch_s / 1e12
+                    / peaks["bf16_tflops"], 4),
+                "roofline_frac": round(max(abytes / (peaks["hbm_gbs"] * 1e9),
+                                           CHUNKED_FLOPS_PER_TOKEN_HEAD * w.B * w.T * w.H
+                                           / (peaks["bf16_tflops"] * 1e12)) / avg_launch_s, 4)}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(lib, G, w, device, stream, (h_q, h_k, h_v, h_g, h_b),
+                      (q, k, v, g, b), out, st_out, world, max(2, min(args.steps, 3)))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, inp, args.cpu_seconds)
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": workload_config(w, layers), "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * layers,
+            "clocks": clock_rec}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+    return line if rank == 0 else None
+
+
+def run_e2e(lib, G, w, device, stream, host_src, dev, out, st_out, world, steps):
+    """The same metric through gdn_forward_host: pinned host inputs copied in,
+    output and final state copied out, every step."""
+    import torch
+    hq, hk, hv, hg, hb = (x.pin_memory() for x in host_src)
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_st = torch.empty(st_out.shape, dtype=torch.float32).pin_memory()
+    q, k, v, g, b = dev
+    sptr = stream.cuda_stream
+
+    def call():
+        st = lib.gdn_forward_host(hq.data_ptr(), hk.data_ptr(), hv.data_ptr(), hg.data_ptr(),
+                                  hb.data_ptr(), None, h_st.data_ptr(), h_out.data_ptr(),
+                                  q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(),
+                                  b.data_ptr(), st_out.data_ptr(), out.data_ptr(),
+                                  w.B, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.chunk_len, sptr)
+        if st != 0:
+            raise G.GdnError(st, "gdn_forward_host")
+
+    call()
+    barrier(world, device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        call()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    elapsed = t0.elapsed_time(t1) / 1e3
+    value, _ = aggregate_throughput(w.B * w.T * steps, elapsed, world, device)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg, hb))
+    d2h = h_out.numel() * h_out.element_size() + h_st.numel() * 4
+    return {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps,
+            "api": "gdn_forward_host (C ABI, pinned host buffers, one layer per step)"}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    from workloads import MINUTE
+    w = MINUTE
+    if args.impl == "reference":
+        line = run_reference(args, w, rank, world)
+    else:
+        line = run_ours(args, w, rank, world, local)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

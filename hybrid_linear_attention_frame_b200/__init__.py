@@ -1,0 +1,15 @@
+"""Frame-wise Gated DeltaNet (GDN) forward pass for SANA-WM on B200 (sm_100a).
+
+The compute lives in ``lib/libgdn.so`` (CUDA, C ABI declared in ``include/gdn.h``);
+``gdn`` is its ctypes binding.
+"""
+
+from .gdn import (GDN_ERR_CUDA, GDN_ERR_INVALID_ARG, GDN_ERR_TIMEOUT, GDN_ERR_UNSUPPORTED, GDN_OK,
+                  GdnError, forward, gdn_bf16_path, gdn_forward, gdn_forward_f32, gdn_forward_host,
+                  gdn_get_last_device_status, gdn_state_step, gdn_state_step_f32, gdn_version,
+                  load, state_step, status_string)
+
+__all__ = ["GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_UNSUPPORTED", "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT",
+           "GdnError", "forward", "state_step", "gdn_forward", "gdn_state_step", "gdn_forward_f32",
+           "gdn_state_step_f32", "gdn_forward_host", "gdn_get_last_device_status", "gdn_bf16_path",
+           "gdn_version", "load", "status_string"]

@@ -1,0 +1,207 @@
+// C ABI of the GDN forward library: argument checks, dispatch, host-buffer entry.
+//
+// Every entry point validates its arguments before touching CUDA and returns a
+// gdn_status; nothing is enqueued on an error.  The library never allocates.
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/gdn.h"
+#include "gdn_common.cuh"
+
+namespace gdn {
+template <typename IOT>
+cudaError_t launch_ffma(const FwdParams& p, int chunk_len, cudaStream_t stream);
+bool tc_supported(int dk, int dv, int chunk_len);
+cudaError_t launch_tc(const FwdParams& p, int chunk_len, cudaStream_t stream);
+int read_and_clear_device_status(cudaStream_t stream);
+}  // namespace gdn
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb)
+{
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t x0 = reinterpret_cast<uintptr_t>(a), y0 = reinterpret_cast<uintptr_t>(b);
+    return x0 < y0 + nb && y0 < x0 + na;
+}
+
+bool supported_dim(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
+
+// Checks shared by every entry point.  `need_out` is false for the
+// state-only streaming step.
+int validate(const void* q, const void* k, const void* v, const float* gate,
+             const float* beta, const float* state_in, const float* state_out,
+             const void* out, bool need_out, size_t elem,
+             int B, int H, int T, int dk, int dv, int frame_len, int chunk_len,
+             gdn::FwdParams* p)
+{
+    if (B < 1 || H < 1 || T < 0 || frame_len < 1) return GDN_ERR_INVALID_ARG;
+    if (dk < 1 || dv < 1 || chunk_len < 1) return GDN_ERR_INVALID_ARG;
+    if (!supported_dim(dk) || !supported_dim(dv)) return GDN_ERR_UNSUPPORTED;
+    if (chunk_len != 16 && chunk_len != 32 && chunk_len != 64) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)B * H > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !gate || !beta) return GDN_ERR_INVALID_ARG;
+    if (need_out && !out) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return GDN_ERR_INVALID_ARG;
+    if (out && !aligned(out, 16)) return GDN_ERR_INVALID_ARG;
+    if ((state_in && !aligned(state_in, 16)) || (state_out && !aligned(state_out, 16)))
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned(gate, 4) || !aligned(beta, 4)) return GDN_ERR_INVALID_ARG;
+
+    const int64_t F = ((int64_t)T + frame_len - 1) / frame_len;
+    const size_t nq = (size_t)B * T * H * dk * elem;
+    const size_t nv = (size_t)B * T * H * dv * elem;
+    const size_t ng = (size_t)B * F * H * sizeof(float);
+    const size_t nb = (size_t)B * T * H * sizeof(float);
+    const size_t ns = (size_t)B * H * dk * dv * sizeof(float);
+    if (out) {
+        if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv) ||
+            overlaps(out, nv, gate, ng) || overlaps(out, nv, beta, nb) ||
+            overlaps(out, nv, state_in, ns) || overlaps(out, nv, state_out, ns))
+            return GDN_ERR_INVALID_ARG;
+    }
+    if (state_out && state_out != state_in) {
+        if (overlaps(state_out, ns, q, nq) || overlaps(state_out, ns, k, nq) ||
+            overlaps(state_out, ns, v, nv) || overlaps(state_out, ns, gate, ng) ||
+            overlaps(state_out, ns, beta, nb) || overlaps(state_out, ns, state_in, ns))
+            return GDN_ERR_INVALID_ARG;
+    }
+    p->q = q; p->k = k; p->v = v; p->gate = gate; p->beta = beta;
+    p->state_in = state_in; p->state_out = const_cast<float*>(state_out);
+    p->out = const_cast<void*>(out);
+    p->B = B; p->H = H; p->T = T; p->dk = dk; p->dv = dv; p->frame_len = frame_len;
+    p->F = (int)F;
+    return GDN_OK;
+}
+
+int to_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+int run_bf16(const gdn::FwdParams& p, int chunk_len, cudaStream_t stream)
+{
+    if (gdn::tc_supported(p.dk, p.dv, chunk_len)) return to_status(gdn::launch_tc(p, chunk_len, stream));
+    return to_status(gdn::launch_ffma<__nv_bfloat16>(p, chunk_len, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_forward(const void* q, const void* k, const void* v,
+                const float* gate_logit, const float* beta_logit,
+                const float* state_in, float* state_out, void* out,
+                int B, int H, int T, int d_k, int d_v,
+                int frame_len, int chunk_len, cudaStream_t stream)
+{
+    gdn::FwdParams p;
+    int st = validate(q, k, v, gate_logit, beta_logit, state_in, state_out, out, true, 2,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
+    if (st != GDN_OK) return st;
+    return run_bf16(p, chunk_len, stream);
+}
+
+int gdn_state_step(const void* q, const void* k, const void* v,
+                   const float* gate_logit, const float* beta_logit,
+                   float* state, void* out,
+                   int B, int H, int T, int d_k, int d_v,
+                   int frame_len, int chunk_len, cudaStream_t stream)
+{
+    if (!state) return GDN_ERR_INVALID_ARG;
+    gdn::FwdParams p;
+    int st = validate(q, k, v, gate_logit, beta_logit, state, state, out, false, 2,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
+    if (st != GDN_OK) return st;
+    return run_bf16(p, chunk_len, stream);
+}
+
+int gdn_forward_f32(const float* q, const float* k, const float* v,
+                    const float* gate_logit, const float* beta_logit,
+                    const float* state_in, float* state_out, float* out,
+                    int B, int H, int T, int d_k, int d_v,
+                    int frame_len, int chunk_len, cudaStream_t stream)
+{
+    gdn::FwdParams p;
+    int st = validate(q, k, v, gate_logit, beta_logit, state_in, state_out, out, true, 4,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
+    if (st != GDN_OK) return st;
+    return to_status(gdn::launch_ffma<float>(p, chunk_len, stream));
+}
+
+int gdn_state_step_f32(const float* q, const float* k, const float* v,
+                       const float* gate_logit, const float* beta_logit,
+                       float* state, float* out,
+                       int B, int H, int T, int d_k, int d_v,
+                       int frame_len, int chunk_len, cudaStream_t stream)
+{
+    if (!state) return GDN_ERR_INVALID_ARG;
+    gdn::FwdParams p;
+    int st = validate(q, k, v, gate_logit, beta_logit, state, state, out, false, 4,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
+    if (st != GDN_OK) return st;
+    return to_status(gdn::launch_ffma<float>(p, chunk_len, stream));
+}
+
+int gdn_forward_host(const void* h_q, const void* h_k, const void* h_v,
+                     const float* h_gate_logit, const float* h_beta_logit,
+                     const float* h_state_in, float* h_state_out, void* h_out,
+                     void* d_q, void* d_k, void* d_v,
+                     float* d_gate_logit, float* d_beta_logit,
+                     float* d_state, void* d_out,
+                     int B, int H, int T, int d_k_dim, int d_v_dim,
+                     int frame_len, int chunk_len, cudaStream_t stream)
+{
+    if (!h_q || !h_k || !h_v || !h_gate_logit || !h_beta_logit || !h_out) return GDN_ERR_INVALID_ARG;
+    if ((h_state_in || h_state_out) && !d_state) return GDN_ERR_INVALID_ARG;
+    gdn::FwdParams p;
+    int st = validate(d_q, d_k, d_v, d_gate_logit, d_beta_logit, h_state_in ? d_state : nullptr,
+                      d_state, d_out, true, 2, B, H, T, d_k_dim, d_v_dim, frame_len,
+                      chunk_len, &p);
+    if (st != GDN_OK) return st;
+    const int64_t F = ((int64_t)T + frame_len - 1) / frame_len;
+    const size_t nq = (size_t)B * T * H * d_k_dim * 2;
+    const size_t nv = (size_t)B * T * H * d_v_dim * 2;
+    const size_t ng = (size_t)B * F * H * sizeof(float);
+    const size_t nb = (size_t)B * T * H * sizeof(float);
+    const size_t ns = (size_t)B * H * d_k_dim * d_v_dim * sizeof(float);
+    cudaError_t e = cudaSuccess;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_q, h_q, nq, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_k, h_k, nq, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_v, h_v, nv, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_gate_logit, h_gate_logit, ng, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_beta_logit, h_beta_logit, nb, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess && h_state_in) e = cudaMemcpyAsync(d_state, h_state_in, ns, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    st = run_bf16(p, chunk_len, stream);
+    if (st != GDN_OK) return st;
+    e = cudaMemcpyAsync(h_out, d_out, nv, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess && h_state_out) e = cudaMemcpyAsync(h_state_out, d_state, ns, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    return to_status(e);
+}
+
+const char* gdn_status_string(int status)
+{
+    switch (status) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument (null, misaligned or overlapping pointer, or bad size)";
+        case GDN_ERR_UNSUPPORTED: return "unsupported size (d_k, d_v in 16..128 step 16; chunk_len 16, 32 or 64)";
+        case GDN_ERR_CUDA: return "CUDA runtime error";
+        case GDN_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int gdn_get_last_device_status(cudaStream_t stream)
+{
+    return gdn::read_and_clear_device_status(stream);
+}
+
+int gdn_bf16_path(int d_k, int d_v, int chunk_len)
+{
+    return gdn::tc_supported(d_k, d_v, chunk_len) ? 1 : 0;
+}
+
+int gdn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,5 @@
+// Single translation unit of libgdn.so: every kernel and the C ABI.
+#include "gdn_status.cu"
+#include "gdn_ffma.cu"
+#include "gdn_tc.cu"
+#include "gdn_api.cu"

@@ -1,0 +1,143 @@
+/*
+ * gdn.h -- C ABI of the frame-wise Gated DeltaNet (GDN) forward pass on B200.
+ *
+ * The operation.  SANA-WM's Stage-1 DiT mixes tokens with "frame-wise Gated
+ * DeltaNet + softmax every 4 blocks" (sglang cookbook SANA-WM page, section 1,
+ * architecture table: 20 heads of head_dim 112) and keeps long causal history
+ * as a bounded recurrent state (same page, introduction; d9249 blog, key-idea
+ * section).  The pages print no formula, so the recurrence is fixed here.  For
+ * every batch entry b and head h independently:
+ *
+ *     S_t = a_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ *   q_t, k_t   L2-normalised per token: x / sqrt(sum_i x_i^2 + 1e-6)
+ *   beta_t     sigmoid(beta_logit[b, t, h])                  (one per token)
+ *   a_t        exp(-softplus(gate_logit[b, t / frame_len, h])) (one per latent
+ *              frame, shared by all frame_len tokens of that frame; token 0 of
+ *              a call is the first token of a frame)
+ *   S          d_k x d_v float32 state (row index = key dimension), carried
+ *              across chunks, frames and calls.
+ *
+ * The kernels evaluate it chunk by chunk (chunk_len tokens) with the WY / UT
+ * form of the delta rule; results equal the token recurrence up to rounding.
+ *
+ * Layouts (row-major, contiguous, element counts):
+ *   q, k        [B, T, H, d_k]     bf16 (gdn_forward / gdn_state_step) or f32 (*_f32)
+ *   v, out      [B, T, H, d_v]     same element type as q
+ *   gate_logit  [B, ceil(T / frame_len), H]  float32
+ *   beta_logit  [B, T, H]          float32
+ *   state       [B, H, d_k, d_v]   float32
+ *
+ * Ownership and memory.  The caller owns every buffer; device pointers must
+ * point to device memory of the current device, host pointers (gdn_forward_host
+ * only) should be pinned.  The library allocates no memory and keeps no state
+ * between calls except one device status word per device.
+ *
+ * Asynchrony.  Work is enqueued on `stream` (0 = legacy default stream) and
+ * the call returns without waiting, except gdn_forward_host, which waits for
+ * its own stream.  Argument errors are reported synchronously and enqueue
+ * nothing.
+ *
+ * Supported sizes: B, H >= 1; T >= 0 (T = 0 passes the state through);
+ * d_k, d_v in {16, 32, ..., 128}; chunk_len in {16, 32, 64}; frame_len >= 1;
+ * B * T * H * max(d_k, d_v) < 2^31 elements per tensor is NOT required (64-bit
+ * indexing), but B * H, T and ceil(T / frame_len) must each fit in an int.
+ * Every pointer to q, k, v, out and the state must be 16-byte aligned; the
+ * logit pointers 4-byte aligned.  `out` must not overlap any input.
+ * state_in == state_out is allowed (in-place update).
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = -1,   /* null / misaligned / overlapping pointer, bad size  */
+    GDN_ERR_UNSUPPORTED = -2,   /* size outside the supported set above               */
+    GDN_ERR_CUDA = -3,          /* a CUDA runtime call or kernel launch failed        */
+    GDN_ERR_TIMEOUT = -4        /* a bounded device-side wait gave up (see below)     */
+} gdn_status;
+
+/*
+ * Forward pass, bf16 q/k/v/out, float32 logits and state.
+ *   state_in   may be NULL: zero initial state.
+ *   state_out  may be NULL: the final state is not written.
+ * Returns a gdn_status.
+ */
+int gdn_forward(const void* q, const void* k, const void* v,
+                const float* gate_logit, const float* beta_logit,
+                const float* state_in, float* state_out, void* out,
+                int B, int H, int T, int d_k, int d_v,
+                int frame_len, int chunk_len, cudaStream_t stream);
+
+/*
+ * One streaming block (SANA-WM streams 3 latent frames per block: sglang
+ * cookbook, section 9 pipeline-config table, num_frame_per_block): advance
+ * the state in place over the block's T tokens.  `state` is read and then
+ * overwritten (must not be NULL); `out` may be NULL (state-only update).
+ */
+int gdn_state_step(const void* q, const void* k, const void* v,
+                   const float* gate_logit, const float* beta_logit,
+                   float* state, void* out,
+                   int B, int H, int T, int d_k, int d_v,
+                   int frame_len, int chunk_len, cudaStream_t stream);
+
+/* float32 reference mode: same operation, float32 q/k/v/out, all-FFMA math. */
+int gdn_forward_f32(const float* q, const float* k, const float* v,
+                    const float* gate_logit, const float* beta_logit,
+                    const float* state_in, float* state_out, float* out,
+                    int B, int H, int T, int d_k, int d_v,
+                    int frame_len, int chunk_len, cudaStream_t stream);
+
+int gdn_state_step_f32(const float* q, const float* k, const float* v,
+                       const float* gate_logit, const float* beta_logit,
+                       float* state, float* out,
+                       int B, int H, int T, int d_k, int d_v,
+                       int frame_len, int chunk_len, cudaStream_t stream);
+
+/*
+ * End-to-end call with HOST buffers (bf16 q/k/v/out, float32 logits/state):
+ * copies the inputs to the caller's device buffers d_* on `stream`, runs
+ * gdn_forward, copies out (and the final state, if h_state_out is not NULL)
+ * back, and waits for the stream.  h_state_in / d_state may be NULL together
+ * (zero initial state); d_state is also where the final state is produced.
+ */
+int gdn_forward_host(const void* h_q, const void* h_k, const void* h_v,
+                     const float* h_gate_logit, const float* h_beta_logit,
+                     const float* h_state_in, float* h_state_out, void* h_out,
+                     void* d_q, void* d_k, void* d_v,
+                     float* d_gate_logit, float* d_beta_logit,
+                     float* d_state, void* d_out,
+                     int B, int H, int T, int d_k_dim, int d_v_dim,
+                     int frame_len, int chunk_len, cudaStream_t stream);
+
+/* Human-readable text of a gdn_status value (static storage). */
+const char* gdn_status_string(int status);
+
+/*
+ * Every wait inside the kernels (on an mbarrier completing a TMA copy or a
+ * tensor-core MMA) is bounded.  A wait that runs out records GDN_ERR_TIMEOUT in
+ * a per-device status word and the kernel stops its work and returns cleanly.
+ * This call synchronises `stream`, returns the recorded status (GDN_OK if none)
+ * and clears it.
+ */
+int gdn_get_last_device_status(cudaStream_t stream);
+
+/* Which kernel the bf16 entry points dispatch to for the given sizes
+ * (0 = FFMA chunked kernel, 1 = tensor-core chunked kernel). */
+int gdn_bf16_path(int d_k, int d_v, int chunk_len);
+
+/* Library version, as major * 10000 + minor * 100 + patch. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -1,0 +1,116 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, and rejects bad arguments synchronously, before any CUDA call.
+
+Fake device addresses are used only for calls that must fail validation; no
+call here reaches a kernel launch.
+"""
+
+import os
+import re
+
+import pytest
+
+import hybrid_linear_attention_frame_b200 as G
+from hybrid_linear_attention_frame_b200 import gdn as B
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "gdn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(gdn_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_loads_and_exports_header_symbols():
+    lib = G.load()
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in gdn.h but not exported"
+    assert set(B.EXPORTS) <= set(names)
+
+
+def test_version_and_status_strings():
+    assert G.gdn_version() >= 100
+    for st in (0, -1, -2, -3, -4):
+        assert G.status_string(st)
+    assert "unknown" in G.status_string(7)
+
+
+A = 1 << 20          # a fake, 16-byte-aligned "device address": never dereferenced
+
+
+def call_fwd(**kw):
+    args = dict(q=A, k=2 * A, v=3 * A, gate=4 * A, beta=5 * A, state_in=None, state_out=None,
+                out=6 * A, B=1, H=2, T=64, dk=32, dv=32, frame_len=16, chunk_len=16)
+    args.update(kw)
+    lib = G.load()
+    return lib.gdn_forward(args["q"], args["k"], args["v"], args["gate"], args["beta"],
+                           args["state_in"], args["state_out"], args["out"], args["B"], args["H"],
+                           args["T"], args["dk"], args["dv"], args["frame_len"],
+                           args["chunk_len"], None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), G.GDN_ERR_INVALID_ARG),
+    (dict(k=None), G.GDN_ERR_INVALID_ARG),
+    (dict(v=None), G.GDN_ERR_INVALID_ARG),
+    (dict(gate=None), G.GDN_ERR_INVALID_ARG),
+    (dict(beta=None), G.GDN_ERR_INVALID_ARG),
+    (dict(out=None), G.GDN_ERR_INVALID_ARG),
+    (dict(B=0), G.GDN_ERR_INVALID_ARG),
+    (dict(H=0), G.GDN_ERR_INVALID_ARG),
+    (dict(T=-1), G.GDN_ERR_INVALID_ARG),
+    (dict(frame_len=0), G.GDN_ERR_INVALID_ARG),
+    (dict(dk=0), G.GDN_ERR_INVALID_ARG),
+    (dict(dk=24), G.GDN_ERR_UNSUPPORTED),
+    (dict(dv=144), G.GDN_ERR_UNSUPPORTED),
+    (dict(dk=8), G.GDN_ERR_UNSUPPORTED),
+    (dict(chunk_len=128), G.GDN_ERR_UNSUPPORTED),
+    (dict(chunk_len=48), G.GDN_ERR_UNSUPPORTED),
+    (dict(q=A + 8), G.GDN_ERR_INVALID_ARG),            # misaligned
+    (dict(out=6 * A + 2), G.GDN_ERR_INVALID_ARG),
+    (dict(state_in=7 * A + 4), G.GDN_ERR_INVALID_ARG),
+    (dict(gate=4 * A + 2), G.GDN_ERR_INVALID_ARG),
+    (dict(out=A + 64), G.GDN_ERR_INVALID_ARG),         # out overlaps q
+    (dict(out=5 * A), G.GDN_ERR_INVALID_ARG),          # out overlaps beta
+    (dict(state_out=A), G.GDN_ERR_INVALID_ARG),        # state_out overlaps q
+])
+def test_forward_rejects_bad_arguments(kw, expect):
+    assert call_fwd(**kw) == expect
+
+
+def test_state_step_requires_state():
+    lib = G.load()
+    st = lib.gdn_state_step(A, 2 * A, 3 * A, 4 * A, 5 * A, None, 6 * A, 1, 2, 64, 32, 32, 16, 16, None)
+    assert st == G.GDN_ERR_INVALID_ARG
+
+
+def test_f32_entry_points_validate_too():
+    lib = G.load()
+    st = lib.gdn_forward_f32(A, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 32, 40,
+                             16, 16, None)
+    assert st == G.GDN_ERR_UNSUPPORTED
+    st = lib.gdn_state_step_f32(A, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 1, 2, 64, 32, 32,
+                                16, 16, None)
+    assert st == G.GDN_ERR_INVALID_ARG
+
+
+def test_host_entry_validates_before_copying():
+    lib = G.load()
+    # missing host output buffer
+    st = lib.gdn_forward_host(A, A, A, A, A, None, None, None, A, 2 * A, 3 * A, 4 * A, 5 * A,
+                              None, 6 * A, 1, 2, 64, 32, 32, 16, 16, None)
+    assert st == G.GDN_ERR_INVALID_ARG
+    # a host state without a device state buffer
+    st = lib.gdn_forward_host(A, A, A, A, A, A, None, A, A, 2 * A, 3 * A, 4 * A, 5 * A,
+                              None, 6 * A, 1, 2, 64, 32, 32, 16, 16, None)
+    assert st == G.GDN_ERR_INVALID_ARG
+
+
+def test_binding_raises_on_error():
+    with pytest.raises(G.GdnError) as e:
+        G.gdn_forward(A, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 24, 32, 16, 16,
+                      stream=0)
+    assert e.value.status == G.GDN_ERR_UNSUPPORTED

@@ -1,0 +1,70 @@
+"""Host logic of bench.py: roofline bookkeeping and the multi-rank aggregation
+(world size 2 over gloo on the CPU, one process per rank)."""
+
+import os
+import socket
+
+import pytest
+
+import bench
+from workloads import MINUTE
+
+
+def test_algorithmic_bytes_is_900_per_token_head():
+    w = MINUTE
+    base = bench.algorithmic_bytes(w, False, False) - w.B * w.n_frames * w.H * 4
+    assert base == 900 * w.B * w.T * w.H
+    st = w.B * w.H * w.d_k * w.d_v * 4
+    assert bench.algorithmic_bytes(w, True, True) == bench.algorithmic_bytes(w, False, False) + 2 * st
+
+
+def test_chunked_flops_constant():
+    C, d = 64, 112
+    assert bench.CHUNKED_FLOPS_PER_TOKEN_HEAD == 10 * C * d + 6 * d * d
+
+
+def test_single_rank_aggregate():
+    v, slowest = bench.aggregate_throughput(1000.0, 0.5, 1)
+    assert v == 2000.0 and slowest == 0.5
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+    bench.dist_init("gloo", world, timeout_s=60)
+    bench.barrier(world)
+    elapsed = 1.0 + rank          # rank 1 is the slowest
+    value, slowest = bench.aggregate_throughput(100.0, elapsed, world)
+    q.put((rank, value, slowest))
+    dist.destroy_process_group()
+
+
+def test_two_rank_gloo_aggregate_takes_slowest_rank():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, value, slowest in res:
+        assert slowest == 2.0                 # max over ranks
+        assert value == pytest.approx(100.0 * 2 / 2.0)
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    args = bench.parse_args(["--impl", "reference"])
+    assert bench.run_reference(args, MINUTE, rank=1, world=2) is None
