@@ -5,7 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
-#include "../../include/gdn.h"
+#include "gdn.h"
 #include "gdn_common.cuh"
 
 namespace gdn {

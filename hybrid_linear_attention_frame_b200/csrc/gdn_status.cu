@@ -1,5 +1,5 @@
 // Per-device status word written by kernels whose bounded waits run out.
-#include "../../include/gdn.h"
+#include "gdn.h"
 #include "gdn_status.cuh"
 
 namespace gdn {

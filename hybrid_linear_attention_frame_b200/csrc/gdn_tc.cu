@@ -1,23 +1,34 @@
 // Tensor-core chunked GDN forward for sm_100a: tcgen05 MMAs with TMEM
-// accumulators, operands staged in shared memory by TMA.
+// accumulators, operands staged in shared memory by TMA, warp-specialised.
 //
 // One CTA owns one (batch, head) chain and 16 columns of the d_k x d_v state
 // (columns evolve independently, so CTAs of a head never communicate).  Per
 // chunk of 64 tokens (notation of gdn_common.cuh):
 //
-//   G1   [K;Q] K^T            M=128 N=64  K=d_k   raw Gram matrices
+//   G1   [K;Q][K;Q]^T         M=128 N=128 K=d_k   raw Gram matrices (diagonal: |k|^2, |q|^2)
 //   ---  A, P from G1 with norms and decay, T = (I+A)^{-1} diag(beta)  (CUDA cores)
 //   WU   [T';T] K , [T';T] V  M=128 N=d_k / 16, K=64   (T' = T diag(e^G / |k|))
 //   MMA1 [Q;W] S              M=128 N=16  K=d_k   -> Q S (raw q) and W S
 //   ---  E = U - W S, E' = diag(e^{G_L-G}/|k|) E  (CUDA cores)
-//   MMA2 K^T E' and [P;T'] E  M=128 N=16  K=64    -> state increment, P E
+//   MMA2 K^T E' and [P;X] E   M=128 N=16  K=64    -> state increment, P E
 //   ---  S <- e^{G_L} S + K^T E' (fp32, registers);  O = diag(e^G/|q|) Q S + P E
 //
 // Every product is one M=128 instruction stream: stacking two 64-row operands
-// ([K;Q], [T';T], [Q;W], [P;T']) fills the 128 TMEM lanes, and each epilogue
-// warp reads only the 32 lanes its warp index may access.  The state is kept
-// in fp32 registers of warps 0-3 (thread m owns row m) for the whole sequence;
-// only its bf16 copy feeds MMA1.
+// ([K;Q], [T';T], [Q;W]) fills the 128 TMEM lanes, and each epilogue warp reads
+// only the 32 lanes its warp index may access.
+//
+// Warp roles.  Only the second half (MMA1, E, MMA2, state) depends on the
+// state; the first half ("prep") depends on the chunk's inputs alone.  Warps
+// 0-3 (chain group) run the state chain of chunk c while warps 4-11 (prep
+// group) prepare chunk c+1, so the two halves overlap.  The state lives in
+// fp32 registers of the chain group (thread m owns row m); only its bf16 copy
+// feeds MMA1.  Each group issues its own MMAs from one warp (warp-uniform
+// operands, elected lane) and waits on its own commit barriers.
+//
+// Hand-offs (mbarriers): tile loads -> prep (tma_full[slot]); prep -> chain
+// (ready[stage]); chain -> prep (stage_free[stage], after the chain has read
+// the stage's P, U and scalars).  Tile slots are refilled by the chain group
+// once MMA2 of the slot's chunk has completed.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include "gdn_common.cuh"
@@ -31,64 +42,78 @@ using namespace sm100;
 
 constexpr int kC = 64;             // chunk length
 constexpr int kVB = 16;            // state columns per CTA
-constexpr int kThreads = 256;      // 8 warps; warp w reads TMEM lanes 32*(w%4) ..
-constexpr int kSlots = 3;          // TMA ring depth (chunks in flight)
+constexpr int kThreads = 384;      // 12 warps; warp w reads TMEM lanes 32*(w%4) ..
+constexpr int kChainThreads = 128; // warps 0-3
+constexpr int kPrepThreads = 256;  // warps 4-11
+constexpr uint32_t kBarChain = 1, kBarPrep = 2;   // named barrier ids
+constexpr int kSlots = 3;          // tile ring depth
 constexpr uint32_t kTmemCols = 512;
 
 // TMEM columns (fp32 accumulators, 128 lanes each)
-constexpr uint32_t kColG = 0;      // [K;Q]K^T      64 columns
-constexpr uint32_t kColW = 64;     // [T';T]K       up to 128 columns
-constexpr uint32_t kColU = 192;    // [T';T]V       16
-constexpr uint32_t kColQW = 208;   // [Q;W]S        16
-constexpr uint32_t kColS = 224;    // K^T E'        16
-constexpr uint32_t kColPE = 240;   // [P;T']E       16
+constexpr uint32_t kColG = 0;      // [K;Q][K;Q]^T    128 columns (prep)
+constexpr uint32_t kColW = 128;    // [T';T]K         up to 128  (prep)
+constexpr uint32_t kColU = 256;    // [T';T]V         2 x 16     (prep -> chain)
+constexpr uint32_t kColQW = 288;   // [Q;W]S          16         (chain)
+constexpr uint32_t kColS = 304;    // K^T E'          16         (chain)
+constexpr uint32_t kColPE = 320;   // [P;X]E          2 x 16     (chain)
 
 // Shared memory (bytes from a 1024-aligned base).  A ring slot holds, for
 // d-columns 0-63 and 64-127 in turn, three consecutive 8 KB SW128 tiles
 // K | Q | W (so that [K;Q] and [Q;W] are 128-row operands), then the V tile.
 constexpr uint32_t kTile = 8192;
 constexpr uint32_t kOffK = 0, kOffQ = kTile, kOffW = 2 * kTile;
-constexpr uint32_t kHalf = 3 * kTile;             // d-columns 64-127
-constexpr uint32_t kOffV = 6 * kTile;             // 64 x 16 bf16, SW32
+constexpr uint32_t kHalf = 3 * kTile;              // d-columns 64-127
+constexpr uint32_t kOffV = 6 * kTile;              // 64 x 16 bf16, SW32
 constexpr uint32_t kSlotBytes = 6 * kTile + 2048;  // 51200
-constexpr uint32_t kOffPTT = kSlots * kSlotBytes;  // P | T' | T  (SW128, 8 KB each)
-constexpr uint32_t kOffAX = kOffPTT + 3 * kTile;   // fp32 [64][65]: A below, (I+A)^-1 above
-constexpr uint32_t kOffMS = kOffAX + 64 * 65 * 4;  // fp32 [32][33] solve scratch
-constexpr uint32_t kOffSc = kOffMS + 32 * 33 * 4;  // per-chunk scalars
-constexpr uint32_t kScFloats = 11 * 64 + 16;
-constexpr uint32_t kOffSB = ((kOffSc + kScFloats * 4 + 255) / 256) * 256;  // S bf16, SW32, 128 rows
-constexpr uint32_t kOffEB = kOffSB + 128 * 32;     // E  bf16, SW32, 64 rows
-constexpr uint32_t kOffEP = kOffEB + 64 * 32;      // E' bf16
+// P[0] | P[1] | T' | T, SW128 tiles of 8 KB.  [P[s]; next tile] is the A operand
+// of P E (its second half only feeds TMEM lanes nobody reads); [T';T] feeds WU.
+constexpr uint32_t kOffPTT = kSlots * kSlotBytes;
+constexpr uint32_t kOffTp = kOffPTT + 2 * kTile;
+constexpr uint32_t kOffT = kOffPTT + 3 * kTile;
+constexpr uint32_t kXS = 68;                        // row stride (floats) of AXI
+// AXI, fp32 [64][68]: (I+A)^{-1} in and below the diagonal (row-major), A
+// transposed strictly above it: A(i, j), j < i, at AXI[j][i].
+constexpr uint32_t kOffAXI = kOffPTT + 4 * kTile;
+constexpr uint32_t kMS = 8;                         // per-warp solve scratch [32][8], kept inside T
+constexpr uint32_t kScFloats = 12 * 64 + 16;
+constexpr uint32_t kOffSc = kOffAXI + 64 * kXS * 4; // scalars[2]
+constexpr uint32_t kOffSB = ((kOffSc + 2 * kScFloats * 4 + 255) / 256) * 256;  // S bf16, SW32
+constexpr uint32_t kOffEB = kOffSB + 128 * 32;      // E  bf16, SW32, 64 rows
+constexpr uint32_t kOffEP = kOffEB + 64 * 32;       // E' bf16
 constexpr uint32_t kOffBar = kOffEP + 64 * 32;
-constexpr uint32_t kNumBars = kSlots + 4;          // tma_full[3], g1, wu, m1, m2
+// barriers: tma_full[3], ready[2], stage_free[2], g1, wu, m1, m2
+constexpr uint32_t kBarTma = 0, kBarReady = 3, kBarFree = 5, kBarG1 = 7, kBarWU = 8, kBarM1 = 9,
+                   kBarM2 = 10, kNumBars = 11;
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
 constexpr uint32_t kSmemUsed = kOffAbort + 4;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for aligning the base
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;   // slack for aligning the base
 
-// scalar table offsets (floats)
+// scalar table offsets (floats) within one stage
 enum : uint32_t {
     SC_G = 0,        // cumulative log-gate G_i
     SC_BETA = 64,    // beta_i (0 beyond the chunk's valid length)
     SC_RK = 128,     // 1 / |k_i|
     SC_RQ = 192,     // 1 / |q_i|
-    SC_GAM = 256,    // e^{G_i}
-    SC_DL = 320,     // e^{G_L - G_i}
-    SC_EXR = 384,    // e^{G_i - G_{16 floor(i/16) - 1}}   (i >= 16)
-    SC_EXC = 448,    // [4][64]: e^{G_{16 b - 1} - G_j}      (j < 16 b)
-    SC_MISC = 704,   // [0] = e^{G_L}
+    SC_GQ = 256,     // e^{G_i} / |q_i|
+    SC_GAM = 320,    // e^{G_i}
+    SC_DL = 384,     // e^{G_L - G_i} / |k_i|   (0 beyond the valid length)
+    SC_EXR = 448,    // e^{G_i - G_{16 floor(i/16) - 1}}   (i >= 16)
+    SC_EXC = 512,    // [4][64]: e^{G_{16 b - 1} - G_j}      (j < 16 b; row 0 unused)
+    SC_MISC = 768,   // [0] = e^{G_L}
 };
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffPTT % 1024 == 0 && kSlotBytes % 1024 == 0, "SW128 tiles need 1024-B alignment");
+static_assert(4 * kMS * 32 * 4 <= kTile, "solve scratch fits in the T tile");
 
-constexpr uint32_t kIdG1 = idesc_bf16(128, 64, false, false);
+constexpr uint32_t kIdG1 = idesc_bf16(128, 128, false, false);
 constexpr uint32_t kIdU = idesc_bf16(128, 16, false, true);
 constexpr uint32_t kIdM1 = idesc_bf16(128, 16, false, true);
 constexpr uint32_t kIdM2S = idesc_bf16(128, 16, true, true);
 constexpr uint32_t kIdM2P = idesc_bf16(128, 16, false, true);
 
-// ---------------------------------------------------------------- MMA issue (one thread)
+// ---------------------------------------------------------------- MMA issue (one warp)
 
 __device__ __forceinline__ uint64_t kmaj128(uint32_t addr) { return smem_desc(addr, 16, 1024, kSwizzle128); }
 __device__ __forceinline__ uint64_t mnmaj128(uint32_t addr) { return smem_desc(addr, kHalf, 1024, kSwizzle128); }
@@ -102,37 +127,40 @@ __device__ __forceinline__ uint32_t dstep(uint32_t tile, int ks) {
 
 __device__ __forceinline__ void issue_g1(uint32_t slot, uint32_t tmem, int nks) {
     for (int ks = 0; ks < nks; ++ks) {
-        const uint32_t a = dstep(slot + kOffK, ks);
-        mma_bf16(tmem + kColG, kmaj128(a), kmaj128(a), kIdG1, ks > 0);
+        const uint64_t a = kmaj128(dstep(slot + kOffK, ks));
+        mma_bf16_warp(tmem + kColG, a, a, kIdG1, ks > 0);
     }
 }
 
-__device__ __forceinline__ void issue_wu(uint32_t slot, uint32_t ptt, uint32_t tmem, int dk) {
+__device__ __forceinline__ void issue_wu(uint32_t slot, uint32_t base, uint32_t tmem, int dk, int s) {
     const uint32_t idw = idesc_bf16(128, dk, false, true);
+#pragma unroll
     for (int ks = 0; ks < kC / 16; ++ks) {
-        const uint64_t a = kmaj128(ptt + kTile + (uint32_t)ks * 32u);      // [T';T]
-        mma_bf16(tmem + kColW, a, mnmaj128(slot + kOffK + (uint32_t)ks * 2048u), idw, ks > 0);
-        mma_bf16(tmem + kColU, a, mnmaj32(slot + kOffV + (uint32_t)ks * 512u), kIdU, ks > 0);
+        const uint64_t a = kmaj128(base + kOffTp + (uint32_t)ks * 32u);      // [T';T]
+        mma_bf16_warp(tmem + kColW, a, mnmaj128(slot + kOffK + (uint32_t)ks * 2048u), idw, ks > 0);
+        mma_bf16_warp(tmem + kColU + 16u * s, a, mnmaj32(slot + kOffV + (uint32_t)ks * 512u), kIdU, ks > 0);
     }
 }
 
 __device__ __forceinline__ void issue_m1(uint32_t slot, uint32_t sb, uint32_t tmem, int nks) {
     for (int ks = 0; ks < nks; ++ks)
-        mma_bf16(tmem + kColQW, kmaj128(dstep(slot + kOffQ, ks)), mnmaj32(sb + (uint32_t)ks * 512u),
-                 kIdM1, ks > 0);
+        mma_bf16_warp(tmem + kColQW, kmaj128(dstep(slot + kOffQ, ks)), mnmaj32(sb + (uint32_t)ks * 512u),
+                      kIdM1, ks > 0);
 }
 
-__device__ __forceinline__ void issue_m2(uint32_t slot, uint32_t ptt, uint32_t eb, uint32_t ep,
-                                         uint32_t tmem) {
+__device__ __forceinline__ void issue_m2(uint32_t slot, uint32_t base, uint32_t eb, uint32_t ep,
+                                         uint32_t tmem, int s) {
+    const uint32_t pa = base + kOffPTT + kTile * (uint32_t)s;
+#pragma unroll
     for (int ks = 0; ks < kC / 16; ++ks) {
-        mma_bf16(tmem + kColS, mnmaj128(slot + kOffK + (uint32_t)ks * 2048u),
-                 mnmaj32(ep + (uint32_t)ks * 512u), kIdM2S, ks > 0);
-        mma_bf16(tmem + kColPE, kmaj128(ptt + (uint32_t)ks * 32u), mnmaj32(eb + (uint32_t)ks * 512u),
-                 kIdM2P, ks > 0);
+        mma_bf16_warp(tmem + kColS, mnmaj128(slot + kOffK + (uint32_t)ks * 2048u),
+                      mnmaj32(ep + (uint32_t)ks * 512u), kIdM2S, ks > 0);
+        mma_bf16_warp(tmem + kColPE + 16u * s, kmaj128(pa + (uint32_t)ks * 32u),
+                      mnmaj32(eb + (uint32_t)ks * 512u), kIdM2P, ks > 0);
     }
 }
 
-// TMA loads of chunk c (tokens c*64 ..) into a ring slot.
+// TMA loads of chunk c (tokens c*64 ..) into a ring slot (one elected lane).
 __device__ __forceinline__ void issue_tma(const CUtensorMap* tq, const CUtensorMap* tk,
                                           const CUtensorMap* tv, uint32_t slot, uint32_t bar,
                                           int c, int h, int b, int vb) {
@@ -145,7 +173,7 @@ __device__ __forceinline__ void issue_tma(const CUtensorMap* tq, const CUtensorM
     tma_load_4d(slot + kOffV, tv, bar, vb * kVB, h, t0, b);
 }
 
-// ---------------------------------------------------------------- epilogue helpers
+// ---------------------------------------------------------------- helpers
 
 // Row `row` of a 16-column bf16 tile in the SW32 layout (two 16-byte chunks).
 __device__ __forceinline__ void store_row16_sw32(uint32_t tile, uint32_t row, const float (&x)[16]) {
@@ -183,68 +211,137 @@ __device__ __forceinline__ float row_sumsq(const uint8_t* row128) {
     return s;
 }
 
+// Group-local barrier that also returns the AND of `v` over the group.
+__device__ __forceinline__ bool group_all(uint32_t id, uint32_t n, bool v) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.u32 p, %3, 0;\n\t"
+                 "bar.red.and.pred q, %1, %2, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"(id), "r"(n), "r"(v ? 1u : 0u) : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void st4(float* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+
 struct TcArgs {
     FwdParams p;
     uint64_t wait_limit_ns;
 };
 
-// (I + A)^{-1} is kept in the upper part of AX: element (i, j), j <= i, at AX[j][i + 1].
-__device__ __forceinline__ float& XI(float* AX, int i, int j) { return AX[j * 65 + i + 1]; }
-__device__ __forceinline__ float AA(const float* AX, int i, int j) { return AX[i * 65 + j]; }
+// ---------------------------------------------------------------- UT inverse
 
-// Blocked inverse of the unit lower-triangular 64x64 matrix I + A (A strictly
-// lower, in AX below the diagonal) by forward substitution on 16x16 diagonal
-// blocks and two levels of block combination
-//   [[X, 0], [C, Y]]^{-1} = [[X^-1, 0], [-Y^-1 C X^-1, Y^-1]].
-// All 256 threads take part; fp32 throughout.
-__device__ void unit_lower_inverse_64(float* AX, float* MS, int tid) {
-    if (tid < 64) {
-        const int o = 16 * (tid >> 4), j = tid & 15;
+// A(i, j) for j < i lives transposed above the diagonal of AXI.
+__device__ __forceinline__ float AAt(const float* AXI, int i, int j) { return AXI[j * kXS + i]; }
+// (I+A)^{-1}(i, j): row-major in and below the diagonal, zero above it.
+__device__ __forceinline__ float XIv(const float* AXI, int i, int j) { return (i >= j) ? AXI[i * kXS + j] : 0.0f; }
+
+__device__ __forceinline__ uint32_t tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// D (16x8) += A (16x8, row) * B (8x8, col), tf32 inputs, fp32 accumulate.  Lane
+// l holds A rows g, g+8 / cols t, t+4; B rows t, t+4 / col g; D rows g, g+8 /
+// cols 2t, 2t+1, with g = l / 4, t = l % 4.
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One 16-row x 8-column tile of  X (rows r0.., K columns c0..) * Y (K rows k0.., 8 columns n0..),
+// X and Y given as element functors, K a multiple of 8.
+template <int K, typename XF, typename YF>
+__device__ __forceinline__ void tile16x8(float (&d)[4], XF X, YF Y, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < K; kk += 8)
+        mma_tf32_16x8x8(d, tf32(X(g, kk + t)), tf32(X(g + 8, kk + t)), tf32(X(g, kk + t + 4)),
+                        tf32(X(g + 8, kk + t + 4)), tf32(Y(kk + t, g)), tf32(Y(kk + t + 4, g)));
+}
+
+// Inverse of the unit lower-triangular 64x64 matrix I + A (A strictly lower,
+// stored transposed above the diagonal of AXI) into the lower triangle of AXI,
+// by forward substitution on the four 16x16 diagonal blocks (fp32 FMA) and two
+// levels of block combination  [[X, 0], [C, Y]]^{-1} = [[X^-1, 0], [-Y^-1 C X^-1, Y^-1]]
+// whose products run on the tensor cores (mma.sync, tf32 in, fp32 accumulate).
+// Every output 8-column tile of a combination depends on the same columns of
+// the intermediate product only, so each warp owns whole column tiles and
+// keeps its intermediate in a private scratch (MSw: [32][8] per warp).
+// Run by the 256 prep threads (pt = 0..255, prep warp pw = pt / 32).
+__device__ void unit_lower_inverse_64(float* AXI, float* MS, int pt) {
+    const int pw = pt >> 5, lane = pt & 31, g = lane >> 2, t = lane & 3;
+    if (pt < 64) {
+        const int o = 16 * (pt >> 4), j = pt & 15;
         float x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             float acc = (i == j) ? 1.0f : 0.0f;
 #pragma unroll
-            for (int m = 0; m < i; ++m) acc = fmaf(-AA(AX, o + i, o + m), x[m], acc);
+            for (int m = 0; m < i; ++m) acc = fmaf(-AAt(AXI, o + i, o + m), x[m], acc);
             x[i] = acc;
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-            if (i >= j) XI(AX, o + i, o + j) = x[i];
+            if (i >= j) AXI[(o + i) * kXS + o + j] = x[i];
     }
-    __syncthreads();
-    // level 1: blocks (1,0) and (3,2)
-    for (int idx = tid; idx < 512; idx += kThreads) {
-        const int pr = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
+    named_bar_sync(kBarPrep, kPrepThreads);
+    float* MSw = MS + pw * 32 * kMS;
+    // level 1: blocks (1,0) and (3,2): Y = -D_hi^{-1} (A_{hi,lo} D_lo^{-1}); warp -> (pair, 8 columns)
+    if (pw < 4) {
+        const int pr = pw >> 1, n0 = 8 * (pw & 1);
         const int hi = 16 * (2 * pr + 1), lo = 16 * (2 * pr);
-        float acc = 0.0f;
-        for (int m = cc; m < 16; ++m) acc = fmaf(AA(AX, hi + r, lo + m), XI(AX, lo + m, lo + cc), acc);
-        MS[(16 * pr + r) * 33 + cc] = acc;
+        float m1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        tile16x8<16>(m1, [&](int r, int k) { return AAt(AXI, hi + r, lo + k); },
+                     [&](int k, int n) { return XIv(AXI, lo + k, lo + n0 + n); }, lane);
+        MSw[g * kMS + 2 * t] = m1[0];
+        MSw[g * kMS + 2 * t + 1] = m1[1];
+        MSw[(g + 8) * kMS + 2 * t] = m1[2];
+        MSw[(g + 8) * kMS + 2 * t + 1] = m1[3];
+        __syncwarp();
+        float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        tile16x8<16>(y, [&](int r, int k) { return XIv(AXI, hi + r, hi + k); },
+                     [&](int k, int n) { return MSw[k * kMS + n]; }, lane);
+        AXI[(hi + g) * kXS + lo + n0 + 2 * t] = -y[0];
+        AXI[(hi + g) * kXS + lo + n0 + 2 * t + 1] = -y[1];
+        AXI[(hi + g + 8) * kXS + lo + n0 + 2 * t] = -y[2];
+        AXI[(hi + g + 8) * kXS + lo + n0 + 2 * t + 1] = -y[3];
     }
-    __syncthreads();
-    for (int idx = tid; idx < 512; idx += kThreads) {
-        const int pr = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
-        const int hi = 16 * (2 * pr + 1), lo = 16 * (2 * pr);
-        float acc = 0.0f;
-        for (int m = 0; m <= r; ++m) acc = fmaf(XI(AX, hi + r, hi + m), MS[(16 * pr + m) * 33 + cc], acc);
-        XI(AX, hi + r, lo + cc) = -acc;
+    named_bar_sync(kBarPrep, kPrepThreads);
+    // level 2: block rows 32-63, columns 0-31; warp -> 8 columns
+    if (pw < 4) {
+        const int n0 = 8 * pw;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            float m2[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            tile16x8<32>(m2, [&](int r, int k) { return AAt(AXI, 32 + 16 * mt + r, k); },
+                         [&](int k, int n) { return XIv(AXI, k, n0 + n); }, lane);
+            MSw[(16 * mt + g) * kMS + 2 * t] = m2[0];
+            MSw[(16 * mt + g) * kMS + 2 * t + 1] = m2[1];
+            MSw[(16 * mt + g + 8) * kMS + 2 * t] = m2[2];
+            MSw[(16 * mt + g + 8) * kMS + 2 * t + 1] = m2[3];
+        }
+        __syncwarp();
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            tile16x8<32>(y, [&](int r, int k) { return XIv(AXI, 32 + 16 * mt + r, 32 + k); },
+                         [&](int k, int n) { return MSw[k * kMS + n]; }, lane);
+            const int r0 = 32 + 16 * mt + g;
+            AXI[r0 * kXS + n0 + 2 * t] = -y[0];
+            AXI[r0 * kXS + n0 + 2 * t + 1] = -y[1];
+            AXI[(r0 + 8) * kXS + n0 + 2 * t] = -y[2];
+            AXI[(r0 + 8) * kXS + n0 + 2 * t + 1] = -y[3];
+        }
     }
-    __syncthreads();
-    // level 2: block rows 32-63, columns 0-31
-    for (int idx = tid; idx < 1024; idx += kThreads) {
-        const int r = idx >> 5, cc = idx & 31;
-        float acc = 0.0f;
-        for (int m = cc; m < 32; ++m) acc = fmaf(AA(AX, 32 + r, m), XI(AX, m, cc), acc);
-        MS[r * 33 + cc] = acc;
-    }
-    __syncthreads();
-    for (int idx = tid; idx < 1024; idx += kThreads) {
-        const int r = idx >> 5, cc = idx & 31;
-        float acc = 0.0f;
-        for (int m = 0; m <= r; ++m) acc = fmaf(XI(AX, 32 + r, 32 + m), MS[m * 33 + cc], acc);
-        XI(AX, 32 + r, cc) = -acc;
-    }
-    __syncthreads();
+    named_bar_sync(kBarPrep, kPrepThreads);
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -263,14 +360,13 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int dk = p.dk, dv = p.dv, nks = dk / 16;
     const int ntk = (p.T + kC - 1) / kC;
 
-    float* AX = reinterpret_cast<float*>(gb + kOffAX);
-    float* MS = reinterpret_cast<float*>(gb + kOffMS);
-    float* sc = reinterpret_cast<float*>(gb + kOffSc);
+    float* AXI = reinterpret_cast<float*>(gb + kOffAXI);
+    float* MSf = reinterpret_cast<float*>(gb + kOffT);
+    float* scal = reinterpret_cast<float*>(gb + kOffSc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + kOffAbort);
-    const uint32_t bar0 = base + kOffBar;
-    const uint32_t bar_g1 = bar0 + 8u * kSlots, bar_wu = bar_g1 + 8u, bar_m1 = bar_g1 + 16u,
-                   bar_m2 = bar_g1 + 24u;
-    const uint32_t ptt = base + kOffPTT, sbt = base + kOffSB, ebt = base + kOffEB, ept = base + kOffEP;
+    const uint32_t bars = base + kOffBar;
+    auto bar = [&](uint32_t i) { return bars + 8u * i; };
+    const uint32_t sbt = base + kOffSB, ebt = base + kOffEB, ept = base + kOffEP;
     const uint64_t lim = args.wait_limit_ns;
     const size_t sbase = ((size_t)b * p.H + h) * (size_t)dk * dv + (size_t)vb * kVB;
 
@@ -279,20 +375,27 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tmem_relinquish();
     }
     if (tid == 32) {
-        for (uint32_t i = 0; i < kNumBars; ++i) mbar_init(bar0 + 8u * i, 1);
+        for (uint32_t i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
         fence_mbar_init();
         *abort_flag = 0;
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
-    // state rows: thread m < 128 of warps 0-3 owns row m of the 16-column slice
+    // chain group: thread m < 128 owns row m of the 16-column state slice
     float S[16];
-    if (tid < 128) {
-        const int m = tid;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            S[j] = (p.state_in && m < dk) ? p.state_in[sbase + (size_t)m * dv + j] : 0.0f;
+    for (int j = 0; j < 16; ++j) S[j] = 0.0f;
+    if (tid < kChainThreads) {
+        const int m = tid;
+        if (p.state_in && m < dk) {
+            const float4* si = reinterpret_cast<const float4*>(p.state_in + sbase + (size_t)m * dv);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float4 v4 = si[j];
+                S[4 * j] = v4.x; S[4 * j + 1] = v4.y; S[4 * j + 2] = v4.z; S[4 * j + 3] = v4.w;
+            }
+        }
         if (m < dk) store_row16_sw32(sbt, (uint32_t)m, S);
     }
     fence_proxy_async_smem();
@@ -300,275 +403,329 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gb + kOffTmemSlot);
-
-    if (tid == 0) {
-        for (int c = 0; c < kSlots - 1 && c < ntk; ++c)
-            issue_tma(&tm_q, &tm_k, &tm_v, base + (uint32_t)c * kSlotBytes, bar0 + 8u * c, c, h, b, vb);
+    int tma_issued = 0;                    // chain warp 0: chunks whose loads were issued
+    if (warp == 0) {
+        tma_issued = min(ntk, kSlots);
+        if (elect_one())
+            for (int c = 0; c < tma_issued; ++c)
+                issue_tma(&tm_q, &tm_k, &tm_v, base + (uint32_t)c * kSlotBytes, bar(kBarTma + c), c, h, b, vb);
+        __syncwarp();
     }
 
-    float QS[16], Ui[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) { QS[j] = 0.0f; Ui[j] = 0.0f; }
     bool ok = true;
-    int c = 0;
-    for (; c < ntk; ++c) {
-        const int s = c % kSlots;
-        const uint32_t slot = base + (uint32_t)s * kSlotBytes;
-        const uint8_t* gslot = gb + (size_t)s * kSlotBytes;
-        const int c0 = c * kC;
-        const int L = min(kC, p.T - c0);
-        const uint32_t ph = (uint32_t)(c & 1);
-
-        if (tid == 0 && c + kSlots - 1 < ntk) {
-            const int cn = c + kSlots - 1;
-            fence_proxy_async_smem();
-            issue_tma(&tm_q, &tm_k, &tm_v, base + (uint32_t)(cn % kSlots) * kSlotBytes,
-                      bar0 + 8u * (cn % kSlots), cn, h, b, vb);
-        }
-
-        // ---- gates: log a per token, inclusive prefix sum over the chunk, beta ----
-        if (warp == 0) {
-            const int i0 = 2 * lane, i1 = i0 + 1;
-            float la0 = 0.0f, la1 = 0.0f, be0 = 0.0f, be1 = 0.0f;
-            if (i0 < L) {
-                const int t = c0 + i0;
-                la0 = -softplus_f(p.gate[((size_t)b * p.F + t / p.frame_len) * p.H + h]);
-                be0 = sigmoid_f(p.beta[((size_t)b * p.T + t) * p.H + h]);
-            }
-            if (i1 < L) {
-                const int t = c0 + i1;
-                la1 = -softplus_f(p.gate[((size_t)b * p.F + t / p.frame_len) * p.H + h]);
-                be1 = sigmoid_f(p.beta[((size_t)b * p.T + t) * p.H + h]);
-            }
-            float x = la0 + la1;
+    if (warp < 4) {
+        // ======================= chain group =======================
+        float QS[16];
+        float gq = 0.0f;                       // e^{G_i} / |q_i| of this thread's output row
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, off);
-                if (lane >= off) x += y;
-            }
-            sc[SC_G + i0] = x - la1;
-            sc[SC_G + i1] = x;
-            sc[SC_BETA + i0] = be0;
-            sc[SC_BETA + i1] = be1;
-        }
-
-        ok = mbar_wait(bar0 + 8u * s, (uint32_t)((c / kSlots) & 1), abort_flag, lim, 1);
-        if (!__syncthreads_and(ok)) break;
-        if (tid == 0) {
-            tc_fence_after();
-            issue_g1(slot, tmem, nks);
-            mma_commit(bar_g1);
-        }
-
-        // ---- norms (2 threads per row: K rows 0-63, Q rows 64-127) and decay tables ----
-        {
-            const int r = tid >> 1, half = tid & 1;
-            const uint8_t* row = gslot + (half ? kHalf : 0u) + (r < 64 ? kOffK : kOffQ) + (uint32_t)(r & 63) * 128u;
-            float ss = row_sumsq(row);
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            if (half == 0) sc[(r < 64 ? SC_RK : SC_RQ) + (r & 63)] = 1.0f / sqrtf(ss + kNormEps);
-        }
-        {
-            const float GL = sc[SC_G + L - 1];
-            if (tid < 64) {
-                const int i = tid;
-                const float Gi = sc[SC_G + i];
-                sc[SC_GAM + i] = expf(Gi);
-                sc[SC_DL + i] = (i < L) ? expf(GL - Gi) : 0.0f;
-                sc[SC_EXR + i] = (i >= 16) ? expf(Gi - sc[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
-                if (i == 0) sc[SC_MISC] = expf(GL);
-            } else {
-                const int idx = tid - 64, bi = 1 + idx / 64, j = idx & 63;
-                sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? expf(sc[SC_G + 16 * bi - 1] - sc[SC_G + j]) : 0.0f;
-            }
-        }
-        __syncthreads();
-
-        // ---- A (fp32, smem) and P (bf16 SW128) from the raw Gram matrices ----
-        ok = mbar_wait(bar_g1, ph, abort_flag, lim, 2);
-        if (!__syncthreads_and(ok)) break;
-        tc_fence_after();
-        {
-            const int ch = warp >> 2;                   // column half: 0-31 or 32-63
-            float v[32];
-            tmem_ld16(tmem_lane(tmem, qtr) + kColG + 32u * ch, *reinterpret_cast<float(*)[16]>(&v[0]));
-            tmem_ld16(tmem_lane(tmem, qtr) + kColG + 32u * ch + 16u, *reinterpret_cast<float(*)[16]>(&v[16]));
+        for (int j = 0; j < 16; ++j) QS[j] = 0.0f;
+        // O = diag(e^G/|q|) Q S + P E for chunk cp (warps 0, 1; rows 32*qtr + lane)
+        auto output = [&](int cp) {
+            if (qtr >= 2) return;
+            const int sp = cp & 1, Lp = min(kC, p.T - cp * kC), i = 32 * qtr + lane;
+            float pe[16];
+            tmem_ld16(tmem_lane(tmem, qtr) + kColPE + 16u * sp, pe);
             tmem_wait_ld();
-            const int i = 32 * (qtr & 1) + lane;        // row within the 64-row matrix
-            const float Gi = sc[SC_G + i], exr = sc[SC_EXR + i];
-            const float* exc = sc + SC_EXC + 64 * (i >> 4);
-            if (qtr < 2) {
-                const float bi = sc[SC_BETA + i] * sc[SC_RK + i];
+            if (i < Lp && p.out) {
+                const float sq = gq;
+                uint32_t w[8];
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int j = 32 * ch + jj;
-                    float a = 0.0f;
-                    if (j < i) {
-                        const float dec = ((j >> 4) == (i >> 4)) ? expf(Gi - sc[SC_G + j]) : exr * exc[j];
-                        a = bi * sc[SC_RK + j] * v[jj] * dec;
-                    }
-                    AX[i * 65 + j] = a;
-                }
-            } else {
-                const float ri = sc[SC_RQ + i];
-                float pv[32];
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int j = 32 * ch + jj;
-                    float pp = 0.0f;
-                    if (j <= i) {
-                        const float dec = ((j >> 4) == (i >> 4)) ? expf(Gi - sc[SC_G + j]) : exr * exc[j];
-                        pp = ri * sc[SC_RK + j] * v[jj] * dec;
-                    }
-                    pv[jj] = pp;
-                }
-#pragma unroll
-                for (int g = 0; g < 4; ++g) store8_sw128(ptt, (uint32_t)i, (uint32_t)(32 * ch + 8 * g), &pv[8 * g]);
+                for (int j = 0; j < 8; ++j)
+                    w[j] = pack_bf16x2(fmaf(sq, QS[2 * j], pe[2 * j]), fmaf(sq, QS[2 * j + 1], pe[2 * j + 1]));
+                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) +
+                                   (((size_t)b * p.T + (size_t)cp * kC + i) * p.H + h) * dv + (size_t)vb * kVB;
+                uint4* o4 = reinterpret_cast<uint4*>(o);
+                o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
             }
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- T = (I + A)^{-1} diag(beta), T' = T diag(e^G / |k|) ----
-        unit_lower_inverse_64(AX, MS, tid);
-        {
-            const int i = tid >> 2, j0 = 16 * (tid & 3);
-            float tv[16], tpv[16];
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-                const int j = j0 + jj;
-                const float x = (j <= i) ? XI(AX, i, j) * sc[SC_BETA + j] : 0.0f;
-                tv[jj] = x;
-                tpv[jj] = x * sc[SC_GAM + j] * sc[SC_RK + j];
-            }
-            store8_sw128(ptt + 2 * kTile, (uint32_t)i, (uint32_t)j0, &tv[0]);
-            store8_sw128(ptt + 2 * kTile, (uint32_t)i, (uint32_t)j0 + 8, &tv[8]);
-            store8_sw128(ptt + kTile, (uint32_t)i, (uint32_t)j0, &tpv[0]);
-            store8_sw128(ptt + kTile, (uint32_t)i, (uint32_t)j0 + 8, &tpv[8]);
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
+        };
+        int c = 0;
+        for (; c < ntk; ++c) {
+            const int s = c & 1;
+            const uint32_t slot = base + (uint32_t)(c % kSlots) * kSlotBytes;
+            const float* sc = scal + s * kScFloats;
+            ok = mbar_wait(bar(kBarReady + s), (uint32_t)((c >> 1) & 1), abort_flag, lim, 6);
+            if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
             tc_fence_after();
-            issue_wu(slot, ptt, tmem, dk);
-            mma_commit(bar_wu);
-        }
-        ok = mbar_wait(bar_wu, ph, abort_flag, lim, 3);
-        if (!__syncthreads_and(ok)) break;
-        tc_fence_after();
-
-        // ---- W (rows in lanes 0-63) to smem next to Q; U (lanes 64-127) to registers ----
-        if (qtr < 2) {
-            const int i = 32 * qtr + lane;
-            const int cbeg = 64 * (warp >> 2);
-            for (int cb = cbeg; cb < cbeg + 64 && cb < dk; cb += 16) {
+            if (warp == 0) {
+                issue_m1(slot, sbt, tmem, nks);
+                mma_commit_warp(bar(kBarM1));
+            }
+            if (c > 0) output(c - 1);          // previous chunk's output while MMA1 runs
+            ok = mbar_wait(bar(kBarM1), (uint32_t)(c & 1), abort_flag, lim, 4);
+            if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
+            tc_fence_after();
+            {
                 float v[16];
-                tmem_ld16(tmem_lane(tmem, qtr) + kColW + (uint32_t)cb, v);
-                tmem_wait_ld();
-                const uint32_t tile = slot + (cb >= 64 ? kHalf : 0u) + kOffW;
-                store8_sw128(tile, (uint32_t)i, (uint32_t)(cb & 63), &v[0]);
-                store8_sw128(tile, (uint32_t)i, (uint32_t)(cb & 63) + 8, &v[8]);
-            }
-        } else if (warp < 4) {
-            tmem_ld16(tmem_lane(tmem, qtr) + kColU, Ui);
-            tmem_wait_ld();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            issue_m1(slot, sbt, tmem, nks);
-            mma_commit(bar_m1);
-        }
-        ok = mbar_wait(bar_m1, ph, abort_flag, lim, 4);
-        if (!__syncthreads_and(ok)) break;
-        tc_fence_after();
-
-        // ---- E = U - W S and E' (warps 2,3); Q S kept by warps 0,1 ----
-        if (warp < 4) {
-            float v[16];
-            tmem_ld16(tmem_lane(tmem, qtr) + kColQW, v);
-            tmem_wait_ld();
-            if (qtr < 2) {
+                tmem_ld16(tmem_lane(tmem, qtr) + kColQW, v);
+                if (qtr < 2) {
+                    gq = sc[SC_GQ + 32 * qtr + lane];
+                    tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) QS[j] = v[j];
+                    for (int j = 0; j < 16; ++j) QS[j] = v[j];
+                } else {
+                    float u[16];
+                    tmem_ld16(tmem_lane(tmem, qtr) + kColU + 16u * s, u);
+                    tmem_wait_ld();
+                    const int i = 32 * (qtr - 2) + lane;
+                    const float d = sc[SC_DL + i];
+                    float e[16], e2[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        e[j] = u[j] - v[j];
+                        e2[j] = e[j] * d;
+                    }
+                    store_row16_sw32(ebt, (uint32_t)i, e);
+                    store_row16_sw32(ept, (uint32_t)i, e2);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(kBarChain, kChainThreads);
+            if (warp == 0) {
+                tc_fence_after();
+                issue_m2(slot, base, ebt, ept, tmem, s);
+                mma_commit_warp(bar(kBarM2));
+            }
+            ok = mbar_wait(bar(kBarM2), (uint32_t)(c & 1), abort_flag, lim, 5);
+            if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
+            tc_fence_after();
+            {
+                const int m = tid;
+                float v[16];
+                tmem_ld16(tmem_lane(tmem, qtr) + kColS, v);
+                tmem_wait_ld();
+                const float gL = sc[SC_MISC];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) S[j] = fmaf(gL, S[j], v[j]);
+                if (m < dk) store_row16_sw32(sbt, (uint32_t)m, S);
+            }
+            // the slot of chunk c is free once MMA2 has read it: refill with chunk c + kSlots
+            if (warp == 0 && c + kSlots < ntk) {
+                if (elect_one()) {
+                    fence_proxy_async_smem();
+                    issue_tma(&tm_q, &tm_k, &tm_v, slot, bar(kBarTma + (c % kSlots)), c + kSlots, h, b, vb);
+                }
+                __syncwarp();
+                tma_issued = c + kSlots + 1;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(kBarChain, kChainThreads);
+            // stage s (P, U, scalars) fully consumed: MMA2 has read P, E read U, S read e^{G_L}
+            if (tid == 0) mbar_arrive(bar(kBarFree + s));
+        }
+        if (ok && ntk > 0) output(ntk - 1);
+        if (!ok && warp == 0) {
+            // drain tile loads still in flight before the shared memory goes away (bounded)
+            if (elect_one()) {
+                for (int cc = max(0, tma_issued - kSlots); cc < tma_issued; ++cc) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!mbar_try_wait(bar(kBarTma + cc % kSlots), (uint32_t)((cc / kSlots) & 1)) &&
+                           globaltimer_ns() - t0 < lim) {
+                    }
+                }
+            }
+            __syncwarp();
+        }
+        if (ok && p.state_out && tid < dk) {
+            float4* so = reinterpret_cast<float4*>(p.state_out + sbase + (size_t)tid * dv);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) so[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+        }
+    } else {
+        // ======================= prep group =======================
+        const int pt = tid - kChainThreads;   // 0..255
+        const int pw = warp - 4;              // 0..7
+        // raw gate / beta logits of tokens 2*lane and 2*lane+1 of chunk cc (prep warp 0)
+        auto load_logits = [&](int cc, float& g0, float& g1, float& r0, float& r1) {
+            const int t0 = cc * kC + 2 * lane, Lc = min(kC, p.T - cc * kC);
+            g0 = g1 = r0 = r1 = 0.0f;
+            if (2 * lane < Lc) {
+                g0 = __ldg(p.gate + ((size_t)b * p.F + t0 / p.frame_len) * p.H + h);
+                r0 = __ldg(p.beta + ((size_t)b * p.T + t0) * p.H + h);
+            }
+            if (2 * lane + 1 < Lc) {
+                g1 = __ldg(p.gate + ((size_t)b * p.F + (t0 + 1) / p.frame_len) * p.H + h);
+                r1 = __ldg(p.beta + ((size_t)b * p.T + t0 + 1) * p.H + h);
+            }
+        };
+        float pg0 = 0.0f, pg1 = 0.0f, pb0 = 0.0f, pb1 = 0.0f;
+        if (pw == 0 && ntk > 0) load_logits(0, pg0, pg1, pb0, pb1);
+        for (int c = 0; c < ntk; ++c) {
+            const int s = c & 1;
+            const uint32_t slot = base + (uint32_t)(c % kSlots) * kSlotBytes;
+            const uint8_t* gslot = gb + (size_t)(c % kSlots) * kSlotBytes;
+            float* sc = scal + s * kScFloats;
+            const int L = min(kC, p.T - c * kC);
+            if (c >= 2) {
+                ok = mbar_wait(bar(kBarFree + s), (uint32_t)(((c - 2) >> 1) & 1), abort_flag, lim, 7);
+                if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            }
+            // ---- gates: log a per token, inclusive prefix sum over the chunk, beta ----
+            if (pw == 0) {
+                const int i0 = 2 * lane, i1 = i0 + 1;
+                const float g0 = pg0, g1 = pg1, r0 = pb0, r1 = pb1;
+                if (c + 1 < ntk) load_logits(c + 1, pg0, pg1, pb0, pb1);
+                const float la0 = (i0 < L) ? -softplus_f(g0) : 0.0f;
+                const float la1 = (i1 < L) ? -softplus_f(g1) : 0.0f;
+                float x = la0 + la1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                sc[SC_G + i0] = x - la1;
+                sc[SC_G + i1] = x;
+                sc[SC_BETA + i0] = (i0 < L) ? sigmoid_f(r0) : 0.0f;
+                sc[SC_BETA + i1] = (i1 < L) ? sigmoid_f(r1) : 0.0f;
+            }
+            ok = mbar_wait(bar(kBarTma + (c % kSlots)), (uint32_t)((c / kSlots) & 1), abort_flag, lim, 1);
+            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            if (pw == 0) {
+                tc_fence_after();
+                issue_g1(slot, tmem, nks);
+                mma_commit_warp(bar(kBarG1));
+            }
+            // ---- decay tables (need only G), computed while G1 runs ----
+            {
+                const float GL = sc[SC_G + L - 1];
+                if (pt < 64) {
+                    const int i = pt;
+                    const float Gi = sc[SC_G + i];
+                    sc[SC_GAM + i] = expf(Gi);
+                    sc[SC_DL + i] = (i < L) ? expf(GL - Gi) : 0.0f;     // times 1/|k_i| below
+                    sc[SC_EXR + i] = (i >= 16) ? expf(Gi - sc[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
+                    if (i == 0) sc[SC_MISC] = expf(GL);
+                } else {
+                    const int idx = pt - 64, bi = 1 + idx / 64, j = idx & 63;
+                    sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? expf(sc[SC_G + 16 * bi - 1] - sc[SC_G + j]) : 0.0f;
+                }
+            }
+            named_bar_sync(kBarPrep, kPrepThreads);
+            ok = mbar_wait(bar(kBarG1), (uint32_t)(c & 1), abort_flag, lim, 2);
+            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            tc_fence_after();
+            // ---- norms from the Gram diagonal: |k_i|^2 (lanes 0-63), |q_i|^2 (lanes 64-127) ----
+            if (pw < 4) {
+                float v[32];
+                tmem_ld16(tmem_lane(tmem, qtr) + kColG + 32u * qtr, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_ld16(tmem_lane(tmem, qtr) + kColG + 32u * qtr + 16u, *reinterpret_cast<float(*)[16]>(&v[16]));
+                tmem_wait_ld();
+                float d = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) d = (j == lane) ? v[j] : d;
+                const float r = 1.0f / sqrtf(d + kNormEps);
+                const int i = 32 * (qtr & 1) + lane;
+                if (qtr < 2) {
+                    sc[SC_RK + i] = r;
+                    sc[SC_DL + i] *= r;
+                } else {
+                    sc[SC_RQ + i] = r;
+                    sc[SC_GQ + i] = r * sc[SC_GAM + i];
+                }
+            }
+            tc_fence_before();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            // ---- A (fp32, transposed into AXI) and P (bf16 SW128) from the raw Gram matrices ----
+            tc_fence_after();
+            if ((qtr & 1) == 0 && (pw >> 2) == 1) {
+                // rows 0-31 x columns 32-63 lie above the diagonal: A has nothing there, P is zero
+                if (qtr == 2) {
+                    const uint32_t ptile = base + kOffPTT + kTile * (uint32_t)s;
+                    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int g8 = 0; g8 < 4; ++g8) store8_sw128(ptile, (uint32_t)lane, (uint32_t)(32 + 8 * g8), z);
+                }
             } else {
-                const int i = 32 * (qtr - 2) + lane;
-                const float sci = sc[SC_DL + i] * sc[SC_RK + i];
-                float e[16], e2[16];
+                const int ch = pw >> 2;                     // column half: 0-31 or 32-63
+                const int i = 32 * (qtr & 1) + lane;        // row within the 64-row matrix
+                const int bi = i >> 4;
+                const float Gi = sc[SC_G + i], exr = sc[SC_EXR + i];
+                const float ri = (qtr < 2) ? sc[SC_BETA + i] * sc[SC_RK + i] : sc[SC_RQ + i];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    e[j] = Ui[j] - v[j];
-                    e2[j] = e[j] * sci;
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int j0 = 32 * ch + 16 * hh;
+                    float v[16], gj[16], rkj[16], ex[16];
+                    tmem_ld16(tmem_lane(tmem, qtr) + kColG + (uint32_t)j0, v);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 a = ld4(sc + SC_G + j0 + 4 * q4);
+                        const float4 r4 = ld4(sc + SC_RK + j0 + 4 * q4);
+                        const float4 e4 = ld4(sc + SC_EXC + 64 * bi + j0 + 4 * q4);
+                        gj[4 * q4] = a.x; gj[4 * q4 + 1] = a.y; gj[4 * q4 + 2] = a.z; gj[4 * q4 + 3] = a.w;
+                        rkj[4 * q4] = r4.x; rkj[4 * q4 + 1] = r4.y; rkj[4 * q4 + 2] = r4.z; rkj[4 * q4 + 3] = r4.w;
+                        ex[4 * q4] = e4.x; ex[4 * q4 + 1] = e4.y; ex[4 * q4 + 2] = e4.z; ex[4 * q4 + 3] = e4.w;
+                    }
+                    tmem_wait_ld();
+                    float val[16];
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int j = j0 + jj;
+                        const float dec = ((j >> 4) == bi) ? __expf(Gi - gj[jj]) : exr * ex[jj];
+                        const bool keep = (qtr < 2) ? (j < i) : (j <= i);
+                        val[jj] = keep ? ri * rkj[jj] * v[jj] * dec : 0.0f;
+                    }
+                    if (qtr < 2) {
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            if (j0 + jj < i) AXI[(j0 + jj) * kXS + i] = val[jj];
+                    } else {
+                        const uint32_t ptile = base + kOffPTT + kTile * (uint32_t)s;
+                        store8_sw128(ptile, (uint32_t)i, (uint32_t)j0, &val[0]);
+                        store8_sw128(ptile, (uint32_t)i, (uint32_t)j0 + 8, &val[8]);
+                    }
                 }
-                store_row16_sw32(ebt, (uint32_t)i, e);
-                store_row16_sw32(ept, (uint32_t)i, e2);
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+            tc_fence_before();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            // ---- T = (I + A)^{-1} diag(beta), T' = T diag(e^G / |k|) ----
+            unit_lower_inverse_64(AXI, MSf, pt);
+            {
+                const int i = pt >> 2, j0 = 16 * (pt & 3);
+                float tv[16], tpv[16];
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int j = j0 + jj;
+                    const float x = (j <= i) ? AXI[i * kXS + j] * sc[SC_BETA + j] : 0.0f;
+                    tv[jj] = x;
+                    tpv[jj] = x * sc[SC_GAM + j] * sc[SC_RK + j];
+                }
+                store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)j0, &tv[0]);
+                store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)j0 + 8, &tv[8]);
+                store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)j0, &tpv[0]);
+                store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)j0 + 8, &tpv[8]);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            if (pw == 0) {
+                tc_fence_after();
+                issue_wu(slot, base, tmem, dk, s);
+                mma_commit_warp(bar(kBarWU));
+            }
+            ok = mbar_wait(bar(kBarWU), (uint32_t)(c & 1), abort_flag, lim, 3);
+            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
             tc_fence_after();
-            issue_m2(slot, ptt, ebt, ept, tmem);
-            mma_commit(bar_m2);
-        }
-        ok = mbar_wait(bar_m2, ph, abort_flag, lim, 5);
-        if (!__syncthreads_and(ok)) break;
-        tc_fence_after();
-
-        // ---- S <- e^{G_L} S + K^T E' ; O = diag(e^G / |q|) Q S + P E ----
-        if (warp < 4) {
-            const int m = tid;
-            float v[16];
-            tmem_ld16(tmem_lane(tmem, qtr) + kColS, v);
-            tmem_wait_ld();
-            const float gL = sc[SC_MISC];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) S[j] = fmaf(gL, S[j], v[j]);
-            if (m < dk) store_row16_sw32(sbt, (uint32_t)m, S);
+            // ---- W (TMEM lanes 0-63) to smem next to Q ----
             if (qtr < 2) {
-                float pe[16];
-                tmem_ld16(tmem_lane(tmem, qtr) + kColPE, pe);
-                tmem_wait_ld();
-                const int i = m;
-                if (i < L && p.out) {
-                    const float sq = sc[SC_GAM + i] * sc[SC_RQ + i];
-                    uint32_t w[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        w[j] = pack_bf16x2(fmaf(sq, QS[2 * j], pe[2 * j]), fmaf(sq, QS[2 * j + 1], pe[2 * j + 1]));
-                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) +
-                                       (((size_t)b * p.T + c0 + i) * p.H + h) * dv + (size_t)vb * kVB;
-                    uint4* o4 = reinterpret_cast<uint4*>(o);
-                    o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                const int i = 32 * qtr + lane;
+                const int cbeg = 64 * (pw >> 2);
+                for (int cb = cbeg; cb < cbeg + 64 && cb < dk; cb += 16) {
+                    float v[16];
+                    tmem_ld16(tmem_lane(tmem, qtr) + kColW + (uint32_t)cb, v);
+                    tmem_wait_ld();
+                    const uint32_t tile = slot + (cb >= 64 ? kHalf : 0u) + kOffW;
+                    store8_sw128(tile, (uint32_t)i, (uint32_t)(cb & 63), &v[0]);
+                    store8_sw128(tile, (uint32_t)i, (uint32_t)(cb & 63) + 8, &v[8]);
                 }
             }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            if (pt == 0) mbar_arrive(bar(kBarReady + s));
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
     }
 
-    if (!ok && tid == 0) {
-        // A bounded wait gave up.  Before the shared memory goes away, wait (again
-        // bounded) for the tile loads still in flight: chunks c .. c + kSlots - 2
-        // were issued and not yet consumed.  MMAs issued before the give-up
-        // complete on their own within microseconds.
-        for (int cc = c; cc < ntk && cc < c + kSlots - 1; ++cc) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(bar0 + 8u * (cc % kSlots), (uint32_t)((cc / kSlots) & 1)) &&
-                   globaltimer_ns() - t0 < lim) {
-            }
-        }
-    }
-    if (ok && p.state_out && tid < 128 && tid < dk) {
-        float4* so = reinterpret_cast<float4*>(p.state_out + sbase + (size_t)tid * dv);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) so[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
-    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
