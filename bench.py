@@ -52,6 +52,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target wall time of the oracle sample")
+    ap.add_argument("--profile-tokens", type=int, default=0,
+                    help="profiling case: two gdn_forward calls on the layer's first T tokens, no timing")
     return ap.parse_args(argv)
 
 
@@ -443,11 +445,37 @@ def run_e2e(lib, G, w, device, stream, host_src, dev, out, st_out, world, steps)
             "api": "gdn_forward_host (C ABI, pinned host buffers, one layer per step)"}
 
 
+def run_profile_case(w, tokens):
+    """Two gdn_forward calls (warm-up + the one a profiler captures) on the first
+    `tokens` tokens of the layer; small enough for a many-pass ncu capture."""
+    import numpy as np
+    import torch
+    import hybrid_linear_attention_frame_b200 as G
+    from workloads import bf16_bits, make_inputs
+    inp = make_inputs(w, T=tokens)
+    def bf16(x):
+        return torch.from_numpy(bf16_bits(x).view(np.int16).copy()).view(torch.bfloat16).cuda()
+    q, k, v = bf16(inp.q), bf16(inp.k), bf16(inp.v)
+    g = torch.from_numpy(inp.gate).cuda()
+    b = torch.from_numpy(inp.beta).cuda()
+    out = torch.empty_like(v)
+    st = torch.empty((w.B, w.H, w.d_k, w.d_v), dtype=torch.float32, device="cuda")
+    for _ in range(2):
+        G.gdn_forward(q, k, v, g, b, None, st, out, w.B, w.H, tokens, w.d_k, w.d_v, w.frame_len,
+                      w.chunk_len)
+    torch.cuda.synchronize()
+    status = G.gdn_get_last_device_status()
+    print(f"profile case: T={tokens}, device status {status}")
+    return 0 if status == G.GDN_OK else 1
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_env()
     from workloads import MINUTE
     w = MINUTE
+    if args.profile_tokens > 0:
+        return run_profile_case(w, args.profile_tokens)
     if args.impl == "reference":
         line = run_reference(args, w, rank, world)
     else:

@@ -45,17 +45,18 @@ constexpr int kVB = 16;            // state columns per CTA
 constexpr int kThreads = 384;      // 12 warps; warp w reads TMEM lanes 32*(w%4) ..
 constexpr int kChainThreads = 128; // warps 0-3
 constexpr int kPrepThreads = 256;  // warps 4-11
-constexpr uint32_t kBarChain = 1, kBarPrep = 2;   // named barrier ids
+constexpr uint32_t kBarChain = 1, kBarPrep = 2, kBarSolve = 3;   // named barrier ids
+constexpr int kSolveThreads = 128; // prep warps 4-7 run the UT inverse
 constexpr int kSlots = 3;          // tile ring depth
 constexpr uint32_t kTmemCols = 512;
 
 // TMEM columns (fp32 accumulators, 128 lanes each)
-constexpr uint32_t kColG = 0;      // [K;Q][K;Q]^T    128 columns (prep)
-constexpr uint32_t kColW = 128;    // [T';T]K         up to 128  (prep)
-constexpr uint32_t kColU = 256;    // [T';T]V         2 x 16     (prep -> chain)
-constexpr uint32_t kColQW = 288;   // [Q;W]S          16         (chain)
-constexpr uint32_t kColS = 304;    // K^T E'          16         (chain)
-constexpr uint32_t kColPE = 320;   // [P;X]E          2 x 16     (chain)
+constexpr uint32_t kColG = 0;      // [K;Q][K;Q]^T    2 x 128 columns (prep, next chunk prefetched)
+constexpr uint32_t kColW = 256;    // [T';T]K         up to 128  (prep)
+constexpr uint32_t kColU = 384;    // [T';T]V         2 x 16     (prep -> chain)
+constexpr uint32_t kColQW = 416;   // [Q;W]S          16         (chain)
+constexpr uint32_t kColS = 432;    // K^T E'          16         (chain)
+constexpr uint32_t kColPE = 448;   // [P;X]E          2 x 16     (chain)
 
 // Shared memory (bytes from a 1024-aligned base).  A ring slot holds, for
 // d-columns 0-63 and 64-127 in turn, three consecutive 8 KB SW128 tiles
@@ -81,9 +82,9 @@ constexpr uint32_t kOffSB = ((kOffSc + 2 * kScFloats * 4 + 255) / 256) * 256;  /
 constexpr uint32_t kOffEB = kOffSB + 128 * 32;      // E  bf16, SW32, 64 rows
 constexpr uint32_t kOffEP = kOffEB + 64 * 32;       // E' bf16
 constexpr uint32_t kOffBar = kOffEP + 64 * 32;
-// barriers: tma_full[3], ready[2], stage_free[2], g1, wu, m1, m2
-constexpr uint32_t kBarTma = 0, kBarReady = 3, kBarFree = 5, kBarG1 = 7, kBarWU = 8, kBarM1 = 9,
-                   kBarM2 = 10, kNumBars = 11;
+// barriers: tma_full[3], ready[2], gates[2], g1[2], wu, m1, m2
+constexpr uint32_t kBarTma = 0, kBarReady = 3, kBarGates = 5, kBarG1 = 7, kBarWU = 9, kBarM1 = 10,
+                   kBarM2 = 11, kNumBars = 12;
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
 constexpr uint32_t kSmemUsed = kOffAbort + 4;
@@ -125,10 +126,10 @@ __device__ __forceinline__ uint32_t dstep(uint32_t tile, int ks) {
     return tile + (ks >= 4 ? kHalf : 0u) + (uint32_t)(ks & 3) * 32u;
 }
 
-__device__ __forceinline__ void issue_g1(uint32_t slot, uint32_t tmem, int nks) {
+__device__ __forceinline__ void issue_g1(uint32_t slot, uint32_t tmem, int nks, int buf) {
     for (int ks = 0; ks < nks; ++ks) {
         const uint64_t a = kmaj128(dstep(slot + kOffK, ks));
-        mma_bf16_warp(tmem + kColG, a, a, kIdG1, ks > 0);
+        mma_bf16_warp(tmem + kColG + 128u * buf, a, a, kIdG1, ks > 0);
     }
 }
 
@@ -275,27 +276,28 @@ __device__ __forceinline__ void tile16x8(float (&d)[4], XF X, YF Y, int lane) {
 // Every output 8-column tile of a combination depends on the same columns of
 // the intermediate product only, so each warp owns whole column tiles and
 // keeps its intermediate in a private scratch (MSw: [32][8] per warp).
-// Run by the 256 prep threads (pt = 0..255, prep warp pw = pt / 32).
-__device__ void unit_lower_inverse_64(float* AXI, float* MS, int pt) {
-    const int pw = pt >> 5, lane = pt & 31, g = lane >> 2, t = lane & 3;
-    if (pt < 64) {
-        const int o = 16 * (pt >> 4), j = pt & 15;
+// Run by the 128 solve threads (st = 0..127, warp pw = st / 32).
+__device__ void unit_lower_inverse_64(float* AXI, float* MS, int st) {
+    const int pw = st >> 5, lane = st & 31, g = lane >> 2, t = lane & 3;
+    if (st < 64) {
+        // column j of the inverse of diagonal block o: right-looking substitution, so
+        // that the updates of step m are independent of each other
+        const int o = 16 * (st >> 4), j = st & 15;
         float x[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float acc = (i == j) ? 1.0f : 0.0f;
+        for (int i = 0; i < 16; ++i) x[i] = (i == j) ? 1.0f : 0.0f;
 #pragma unroll
-            for (int m = 0; m < i; ++m) acc = fmaf(-AAt(AXI, o + i, o + m), x[m], acc);
-            x[i] = acc;
-        }
+        for (int m = 0; m < 15; ++m)
+#pragma unroll
+            for (int i = m + 1; i < 16; ++i) x[i] = fmaf(-AAt(AXI, o + i, o + m), x[m], x[i]);
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             if (i >= j) AXI[(o + i) * kXS + o + j] = x[i];
     }
-    named_bar_sync(kBarPrep, kPrepThreads);
+    named_bar_sync(kBarSolve, kSolveThreads);
     float* MSw = MS + pw * 32 * kMS;
     // level 1: blocks (1,0) and (3,2): Y = -D_hi^{-1} (A_{hi,lo} D_lo^{-1}); warp -> (pair, 8 columns)
-    if (pw < 4) {
+    {
         const int pr = pw >> 1, n0 = 8 * (pw & 1);
         const int hi = 16 * (2 * pr + 1), lo = 16 * (2 * pr);
         float m1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -314,9 +316,9 @@ __device__ void unit_lower_inverse_64(float* AXI, float* MS, int pt) {
         AXI[(hi + g + 8) * kXS + lo + n0 + 2 * t] = -y[2];
         AXI[(hi + g + 8) * kXS + lo + n0 + 2 * t + 1] = -y[3];
     }
-    named_bar_sync(kBarPrep, kPrepThreads);
+    named_bar_sync(kBarSolve, kSolveThreads);
     // level 2: block rows 32-63, columns 0-31; warp -> 8 columns
-    if (pw < 4) {
+    {
         const int n0 = 8 * pw;
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
@@ -341,7 +343,7 @@ __device__ void unit_lower_inverse_64(float* AXI, float* MS, int pt) {
             AXI[(r0 + 8) * kXS + n0 + 2 * t + 1] = -y[3];
         }
     }
-    named_bar_sync(kBarPrep, kPrepThreads);
+    named_bar_sync(kBarSolve, kSolveThreads);
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -419,6 +421,60 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         float gq = 0.0f;                       // e^{G_i} / |q_i| of this thread's output row
 #pragma unroll
         for (int j = 0; j < 16; ++j) QS[j] = 0.0f;
+        // raw gate / beta logits of tokens 2*lane and 2*lane+1 of chunk cc (warp 0)
+        auto load_logits = [&](int cc, float& g0, float& g1, float& r0, float& r1) {
+            const int t0 = cc * kC + 2 * lane, Lc = min(kC, p.T - cc * kC);
+            g0 = g1 = r0 = r1 = 0.0f;
+            if (2 * lane < Lc) {
+                g0 = __ldg(p.gate + ((size_t)b * p.F + t0 / p.frame_len) * p.H + h);
+                r0 = __ldg(p.beta + ((size_t)b * p.T + t0) * p.H + h);
+            }
+            if (2 * lane + 1 < Lc) {
+                g1 = __ldg(p.gate + ((size_t)b * p.F + (t0 + 1) / p.frame_len) * p.H + h);
+                r1 = __ldg(p.beta + ((size_t)b * p.T + t0 + 1) * p.H + h);
+            }
+        };
+        float pg0 = 0.0f, pg1 = 0.0f, pb0 = 0.0f, pb1 = 0.0f;
+        if (warp == 0 && ntk > 0) load_logits(0, pg0, pg1, pb0, pb1);
+        // Gates and decay tables of chunk cc into stage cc & 1 (whose previous chunk
+        // the chain has finished), then release them to the prep group.
+        auto compute_gates = [&](int cc) {
+            float* sc = scal + (cc & 1) * kScFloats;
+            const int L = min(kC, p.T - cc * kC);
+            if (warp == 0) {
+                const int i0 = 2 * lane, i1 = i0 + 1;
+                const float g0 = pg0, g1 = pg1, r0 = pb0, r1 = pb1;
+                if (cc + 1 < ntk) load_logits(cc + 1, pg0, pg1, pb0, pb1);
+                const float la0 = (i0 < L) ? -softplus_f(g0) : 0.0f;
+                const float la1 = (i1 < L) ? -softplus_f(g1) : 0.0f;
+                float x = la0 + la1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                sc[SC_G + i0] = x - la1;
+                sc[SC_G + i1] = x;
+                sc[SC_BETA + i0] = (i0 < L) ? sigmoid_f(r0) : 0.0f;
+                sc[SC_BETA + i1] = (i1 < L) ? sigmoid_f(r1) : 0.0f;
+            }
+            named_bar_sync(kBarChain, kChainThreads);
+            const float GL = sc[SC_G + L - 1];
+            if (tid < 64) {
+                const int i = tid;
+                const float Gi = sc[SC_G + i];
+                sc[SC_GAM + i] = expf(Gi);
+                sc[SC_DL + i] = (i < L) ? expf(GL - Gi) : 0.0f;     // times 1/|k_i| in the prep
+                sc[SC_EXR + i] = (i >= 16) ? expf(Gi - sc[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
+                if (i == 0) sc[SC_MISC] = expf(GL);
+            }
+            for (int idx = tid; idx < 192; idx += kChainThreads) {
+                const int bi = 1 + idx / 64, j = idx & 63;
+                sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? expf(sc[SC_G + 16 * bi - 1] - sc[SC_G + j]) : 0.0f;
+            }
+            named_bar_sync(kBarChain, kChainThreads);
+            if (tid == 0) mbar_arrive(bar(kBarGates + (cc & 1)));
+        };
         // O = diag(e^G/|q|) Q S + P E for chunk cp (warps 0, 1; rows 32*qtr + lane)
         auto output = [&](int cp) {
             if (qtr >= 2) return;
@@ -439,11 +495,13 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
             }
         };
+        if (ntk > 0) compute_gates(0);
         int c = 0;
         for (; c < ntk; ++c) {
             const int s = c & 1;
             const uint32_t slot = base + (uint32_t)(c % kSlots) * kSlotBytes;
             const float* sc = scal + s * kScFloats;
+            if (c + 1 < ntk) compute_gates(c + 1);
             ok = mbar_wait(bar(kBarReady + s), (uint32_t)((c >> 1) & 1), abort_flag, lim, 6);
             if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
             tc_fence_after();
@@ -512,8 +570,6 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(kBarChain, kChainThreads);
-            // stage s (P, U, scalars) fully consumed: MMA2 has read P, E read U, S read e^{G_L}
-            if (tid == 0) mbar_arrive(bar(kBarFree + s));
         }
         if (ok && ntk > 0) output(ntk - 1);
         if (!ok && warp == 0) {
@@ -537,80 +593,34 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // ======================= prep group =======================
         const int pt = tid - kChainThreads;   // 0..255
         const int pw = warp - 4;              // 0..7
-        // raw gate / beta logits of tokens 2*lane and 2*lane+1 of chunk cc (prep warp 0)
-        auto load_logits = [&](int cc, float& g0, float& g1, float& r0, float& r1) {
-            const int t0 = cc * kC + 2 * lane, Lc = min(kC, p.T - cc * kC);
-            g0 = g1 = r0 = r1 = 0.0f;
-            if (2 * lane < Lc) {
-                g0 = __ldg(p.gate + ((size_t)b * p.F + t0 / p.frame_len) * p.H + h);
-                r0 = __ldg(p.beta + ((size_t)b * p.T + t0) * p.H + h);
-            }
-            if (2 * lane + 1 < Lc) {
-                g1 = __ldg(p.gate + ((size_t)b * p.F + (t0 + 1) / p.frame_len) * p.H + h);
-                r1 = __ldg(p.beta + ((size_t)b * p.T + t0 + 1) * p.H + h);
-            }
-        };
-        float pg0 = 0.0f, pg1 = 0.0f, pb0 = 0.0f, pb1 = 0.0f;
-        if (pw == 0 && ntk > 0) load_logits(0, pg0, pg1, pb0, pb1);
-        for (int c = 0; c < ntk; ++c) {
-            const int s = c & 1;
-            const uint32_t slot = base + (uint32_t)(c % kSlots) * kSlotBytes;
-            const uint8_t* gslot = gb + (size_t)(c % kSlots) * kSlotBytes;
-            float* sc = scal + s * kScFloats;
-            const int L = min(kC, p.T - c * kC);
-            if (c >= 2) {
-                ok = mbar_wait(bar(kBarFree + s), (uint32_t)(((c - 2) >> 1) & 1), abort_flag, lim, 7);
-                if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
-            }
-            // ---- gates: log a per token, inclusive prefix sum over the chunk, beta ----
-            if (pw == 0) {
-                const int i0 = 2 * lane, i1 = i0 + 1;
-                const float g0 = pg0, g1 = pg1, r0 = pb0, r1 = pb1;
-                if (c + 1 < ntk) load_logits(c + 1, pg0, pg1, pb0, pb1);
-                const float la0 = (i0 < L) ? -softplus_f(g0) : 0.0f;
-                const float la1 = (i1 < L) ? -softplus_f(g1) : 0.0f;
-                float x = la0 + la1;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, off);
-                    if (lane >= off) x += y;
-                }
-                sc[SC_G + i0] = x - la1;
-                sc[SC_G + i1] = x;
-                sc[SC_BETA + i0] = (i0 < L) ? sigmoid_f(r0) : 0.0f;
-                sc[SC_BETA + i1] = (i1 < L) ? sigmoid_f(r1) : 0.0f;
-            }
-            ok = mbar_wait(bar(kBarTma + (c % kSlots)), (uint32_t)((c / kSlots) & 1), abort_flag, lim, 1);
-            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
-            if (pw == 0) {
+        // G1 of chunk cc into accumulator buffer cc & 1, issued by prep warp 4 (not in the solve)
+        auto prefetch_g1 = [&](int cc) -> bool {
+            const bool got = mbar_wait(bar(kBarTma + (cc % kSlots)), (uint32_t)((cc / kSlots) & 1),
+                                       abort_flag, lim, 1);
+            if (got) {
                 tc_fence_after();
-                issue_g1(slot, tmem, nks);
-                mma_commit_warp(bar(kBarG1));
+                issue_g1(base + (uint32_t)(cc % kSlots) * kSlotBytes, tmem, nks, cc & 1);
+                mma_commit_warp(bar(kBarG1 + (cc & 1)));
             }
-            // ---- decay tables (need only G), computed while G1 runs ----
-            {
-                const float GL = sc[SC_G + L - 1];
-                if (pt < 64) {
-                    const int i = pt;
-                    const float Gi = sc[SC_G + i];
-                    sc[SC_GAM + i] = expf(Gi);
-                    sc[SC_DL + i] = (i < L) ? expf(GL - Gi) : 0.0f;     // times 1/|k_i| below
-                    sc[SC_EXR + i] = (i >= 16) ? expf(Gi - sc[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
-                    if (i == 0) sc[SC_MISC] = expf(GL);
-                } else {
-                    const int idx = pt - 64, bi = 1 + idx / 64, j = idx & 63;
-                    sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? expf(sc[SC_G + 16 * bi - 1] - sc[SC_G + j]) : 0.0f;
-                }
-            }
-            named_bar_sync(kBarPrep, kPrepThreads);
-            ok = mbar_wait(bar(kBarG1), (uint32_t)(c & 1), abort_flag, lim, 2);
+            return got;
+        };
+        bool pre_ok = true;
+        if (pw == 4 && ntk > 0) pre_ok = prefetch_g1(0);
+        for (int c = 0; c < ntk; ++c) {
+            const int s = c & 1, gbuf = c & 1;
+            const uint32_t slot = base + (uint32_t)(c % kSlots) * kSlotBytes;
+            float* sc = scal + s * kScFloats;
+            ok = pre_ok && mbar_wait(bar(kBarGates + s), (uint32_t)((c >> 1) & 1), abort_flag, lim, 7);
+            ok = ok && mbar_wait(bar(kBarTma + (c % kSlots)), (uint32_t)((c / kSlots) & 1), abort_flag, lim, 1);
+            ok = ok && mbar_wait(bar(kBarG1 + gbuf), (uint32_t)((c >> 1) & 1), abort_flag, lim, 2);
             if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
             tc_fence_after();
+            const uint32_t tg = tmem + kColG + 128u * gbuf;
             // ---- norms from the Gram diagonal: |k_i|^2 (lanes 0-63), |q_i|^2 (lanes 64-127) ----
             if (pw < 4) {
                 float v[32];
-                tmem_ld16(tmem_lane(tmem, qtr) + kColG + 32u * qtr, *reinterpret_cast<float(*)[16]>(&v[0]));
-                tmem_ld16(tmem_lane(tmem, qtr) + kColG + 32u * qtr + 16u, *reinterpret_cast<float(*)[16]>(&v[16]));
+                tmem_ld16(tmem_lane(tg, qtr) + 32u * qtr, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_ld16(tmem_lane(tg, qtr) + 32u * qtr + 16u, *reinterpret_cast<float(*)[16]>(&v[16]));
                 tmem_wait_ld();
                 float d = 0.0f;
 #pragma unroll
@@ -625,10 +635,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     sc[SC_GQ + i] = r * sc[SC_GAM + i];
                 }
             }
-            tc_fence_before();
             named_bar_sync(kBarPrep, kPrepThreads);
             // ---- A (fp32, transposed into AXI) and P (bf16 SW128) from the raw Gram matrices ----
-            tc_fence_after();
             if ((qtr & 1) == 0 && (pw >> 2) == 1) {
                 // rows 0-31 x columns 32-63 lie above the diagonal: A has nothing there, P is zero
                 if (qtr == 2) {
@@ -647,7 +655,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int hh = 0; hh < 2; ++hh) {
                     const int j0 = 32 * ch + 16 * hh;
                     float v[16], gj[16], rkj[16], ex[16];
-                    tmem_ld16(tmem_lane(tmem, qtr) + kColG + (uint32_t)j0, v);
+                    tmem_ld16(tmem_lane(tg, qtr) + (uint32_t)j0, v);
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         const float4 a = ld4(sc + SC_G + j0 + 4 * q4);
@@ -679,25 +687,32 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc_fence_before();
             named_bar_sync(kBarPrep, kPrepThreads);
-            // ---- T = (I + A)^{-1} diag(beta), T' = T diag(e^G / |k|) ----
-            unit_lower_inverse_64(AXI, MSf, pt);
-            {
-                const int i = pt >> 2, j0 = 16 * (pt & 3);
-                float tv[16], tpv[16];
+            bool ok2 = true;
+            if (pw == 4) {
+                // next chunk's Gram matrices run on the tensor cores during this chunk's solve
+                if (c + 1 < ntk) ok2 = prefetch_g1(c + 1);
+            } else if (pw < 4) {
+                // ---- T = (I + A)^{-1} diag(beta), T' = T diag(e^G / |k|) ----
+                unit_lower_inverse_64(AXI, MSf, pt);
+                const int i = pt >> 1, j0 = 32 * (pt & 1);
 #pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                    const int j = j0 + jj;
-                    const float x = (j <= i) ? AXI[i * kXS + j] * sc[SC_BETA + j] : 0.0f;
-                    tv[jj] = x;
-                    tpv[jj] = x * sc[SC_GAM + j] * sc[SC_RK + j];
+                for (int q = 0; q < 2; ++q) {
+                    float tv[16], tpv[16];
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int j = j0 + 16 * q + jj;
+                        const float x = (j <= i) ? AXI[i * kXS + j] * sc[SC_BETA + j] : 0.0f;
+                        tv[jj] = x;
+                        tpv[jj] = x * sc[SC_GAM + j] * sc[SC_RK + j];
+                    }
+                    store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)(j0 + 16 * q), &tv[0]);
+                    store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)(j0 + 16 * q + 8), &tv[8]);
+                    store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)(j0 + 16 * q), &tpv[0]);
+                    store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)(j0 + 16 * q + 8), &tpv[8]);
                 }
-                store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)j0, &tv[0]);
-                store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)j0 + 8, &tv[8]);
-                store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)j0, &tpv[0]);
-                store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)j0 + 8, &tpv[8]);
             }
             fence_proxy_async_smem();
-            named_bar_sync(kBarPrep, kPrepThreads);
+            if (!group_all(kBarPrep, kPrepThreads, ok2)) { ok = false; break; }
             if (pw == 0) {
                 tc_fence_after();
                 issue_wu(slot, base, tmem, dk, s);
@@ -723,6 +738,14 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_before();
             named_bar_sync(kBarPrep, kPrepThreads);
             if (pt == 0) mbar_arrive(bar(kBarReady + s));
+        }
+        if (!ok && pw == 4) {
+            // a Gram MMA may still be in flight: wait for it (bounded) before TMEM is freed
+            const uint64_t t0 = globaltimer_ns();
+            for (int bb = 0; bb < 2; ++bb)
+                while (!mbar_try_wait(bar(kBarG1 + bb), 0) && !mbar_try_wait(bar(kBarG1 + bb), 1) &&
+                       globaltimer_ns() - t0 < lim) {
+                }
         }
     }
 
