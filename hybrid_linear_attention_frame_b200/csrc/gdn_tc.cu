@@ -76,7 +76,7 @@ constexpr uint32_t kXS = 68;                        // row stride (floats) of AX
 // transposed strictly above it: A(i, j), j < i, at AXI[j][i].
 constexpr uint32_t kOffAXI = kOffPTT + 4 * kTile;
 constexpr uint32_t kMS = 8;                         // per-warp solve scratch [32][8], kept inside T
-constexpr uint32_t kScFloats = 12 * 64 + 16;
+constexpr uint32_t kScFloats = 13 * 64 + 16;
 constexpr uint32_t kOffSc = kOffAXI + 64 * kXS * 4; // scalars[2]
 constexpr uint32_t kOffSB = ((kOffSc + 2 * kScFloats * 4 + 255) / 256) * 256;  // S bf16, SW32
 constexpr uint32_t kOffEB = kOffSB + 128 * 32;      // E  bf16, SW32, 64 rows
@@ -101,7 +101,8 @@ enum : uint32_t {
     SC_DL = 384,     // e^{G_L - G_i} / |k_i|   (0 beyond the valid length)
     SC_EXR = 448,    // e^{G_i - G_{16 floor(i/16) - 1}}   (i >= 16)
     SC_EXC = 512,    // [4][64]: e^{G_{16 b - 1} - G_j}      (j < 16 b; row 0 unused)
-    SC_MISC = 768,   // [0] = e^{G_L}
+    SC_BGK = 768,    // beta_j e^{G_j} / |k_j|
+    SC_MISC = 832,   // [0] = e^{G_L}
 };
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -175,6 +176,14 @@ __device__ __forceinline__ void issue_tma(const CUtensorMap* tq, const CUtensorM
 }
 
 // ---------------------------------------------------------------- helpers
+
+// Gates with the hardware exp2/log2 approximations (results feed bf16 outputs).
+__device__ __forceinline__ float softplus_fast(float x) {
+    return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x)));
+}
+__device__ __forceinline__ float sigmoid_fast(float x) {
+    return __fdividef(1.0f, 1.0f + __expf(-x));
+}
 
 // Row `row` of a 16-column bf16 tile in the SW32 layout (two 16-byte chunks).
 __device__ __forceinline__ void store_row16_sw32(uint32_t tile, uint32_t row, const float (&x)[16]) {
@@ -445,8 +454,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int i0 = 2 * lane, i1 = i0 + 1;
                 const float g0 = pg0, g1 = pg1, r0 = pb0, r1 = pb1;
                 if (cc + 1 < ntk) load_logits(cc + 1, pg0, pg1, pb0, pb1);
-                const float la0 = (i0 < L) ? -softplus_f(g0) : 0.0f;
-                const float la1 = (i1 < L) ? -softplus_f(g1) : 0.0f;
+                const float la0 = (i0 < L) ? -softplus_fast(g0) : 0.0f;
+                const float la1 = (i1 < L) ? -softplus_fast(g1) : 0.0f;
                 float x = la0 + la1;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
@@ -455,22 +464,22 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 sc[SC_G + i0] = x - la1;
                 sc[SC_G + i1] = x;
-                sc[SC_BETA + i0] = (i0 < L) ? sigmoid_f(r0) : 0.0f;
-                sc[SC_BETA + i1] = (i1 < L) ? sigmoid_f(r1) : 0.0f;
+                sc[SC_BETA + i0] = (i0 < L) ? sigmoid_fast(r0) : 0.0f;
+                sc[SC_BETA + i1] = (i1 < L) ? sigmoid_fast(r1) : 0.0f;
             }
             named_bar_sync(kBarChain, kChainThreads);
             const float GL = sc[SC_G + L - 1];
             if (tid < 64) {
                 const int i = tid;
                 const float Gi = sc[SC_G + i];
-                sc[SC_GAM + i] = expf(Gi);
-                sc[SC_DL + i] = (i < L) ? expf(GL - Gi) : 0.0f;     // times 1/|k_i| in the prep
-                sc[SC_EXR + i] = (i >= 16) ? expf(Gi - sc[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
-                if (i == 0) sc[SC_MISC] = expf(GL);
+                sc[SC_GAM + i] = __expf(Gi);
+                sc[SC_DL + i] = (i < L) ? __expf(GL - Gi) : 0.0f;     // times 1/|k_i| in the prep
+                sc[SC_EXR + i] = (i >= 16) ? __expf(Gi - sc[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
+                if (i == 0) sc[SC_MISC] = __expf(GL);
             }
             for (int idx = tid; idx < 192; idx += kChainThreads) {
                 const int bi = 1 + idx / 64, j = idx & 63;
-                sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? expf(sc[SC_G + 16 * bi - 1] - sc[SC_G + j]) : 0.0f;
+                sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? __expf(sc[SC_G + 16 * bi - 1] - sc[SC_G + j]) : 0.0f;
             }
             named_bar_sync(kBarChain, kChainThreads);
             if (tid == 0) mbar_arrive(bar(kBarGates + (cc & 1)));
@@ -625,11 +634,12 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 float d = 0.0f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) d = (j == lane) ? v[j] : d;
-                const float r = 1.0f / sqrtf(d + kNormEps);
+                const float r = rsqrtf(d + kNormEps);
                 const int i = 32 * (qtr & 1) + lane;
                 if (qtr < 2) {
                     sc[SC_RK + i] = r;
                     sc[SC_DL + i] *= r;
+                    sc[SC_BGK + i] = sc[SC_BETA + i] * sc[SC_GAM + i] * r;
                 } else {
                     sc[SC_RQ + i] = r;
                     sc[SC_GQ + i] = r * sc[SC_GAM + i];
@@ -697,18 +707,27 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int i = pt >> 1, j0 = 32 * (pt & 1);
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
+                    const int jb = j0 + 16 * q;
                     float tv[16], tpv[16];
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int j = j0 + 16 * q + jj;
-                        const float x = (j <= i) ? AXI[i * kXS + j] * sc[SC_BETA + j] : 0.0f;
-                        tv[jj] = x;
-                        tpv[jj] = x * sc[SC_GAM + j] * sc[SC_RK + j];
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 x4 = ld4(AXI + i * kXS + jb + 4 * q4);
+                        const float4 b4 = ld4(sc + SC_BETA + jb + 4 * q4);
+                        const float4 f4 = ld4(sc + SC_BGK + jb + 4 * q4);
+                        const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+                        const float bs[4] = {b4.x, b4.y, b4.z, b4.w};
+                        const float fs[4] = {f4.x, f4.y, f4.z, f4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float x = (jb + 4 * q4 + e <= i) ? xs[e] : 0.0f;
+                            tv[4 * q4 + e] = x * bs[e];
+                            tpv[4 * q4 + e] = x * fs[e];
+                        }
                     }
-                    store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)(j0 + 16 * q), &tv[0]);
-                    store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)(j0 + 16 * q + 8), &tv[8]);
-                    store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)(j0 + 16 * q), &tpv[0]);
-                    store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)(j0 + 16 * q + 8), &tpv[8]);
+                    store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)jb, &tv[0]);
+                    store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)jb + 8, &tv[8]);
+                    store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)jb, &tpv[0]);
+                    store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)jb + 8, &tpv[8]);
                 }
             }
             fence_proxy_async_smem();
