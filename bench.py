@@ -36,9 +36,11 @@ METRIC = "GDN fwd tokens/s per layer (20 heads x d112) on 1 B200; % of roofline"
 UNIT = "tokens/s"
 BYTES_PER_TOKEN_HEAD = 900          # q, k, v in + out (bf16, d = 112) + beta logit (f32)
 CHUNKED_FLOPS_PER_TOKEN_HEAD = 146944   # 10 C d + 6 d^2 at C = 64, d = 112
-KERNEL_SOURCES = ["hybrid_linear_attention_frame_b200/csrc/gdn_tc.cu",
+KERNEL_SOURCES = ["hybrid_linear_attention_frame_b200/csrc/gdn_ring.cu",
+                  "hybrid_linear_attention_frame_b200/csrc/gdn_tc.cu",
                   "hybrid_linear_attention_frame_b200/csrc/gdn_ffma.cu",
-                  "hybrid_linear_attention_frame_b200/csrc/gdn_common.cuh"]
+                  "hybrid_linear_attention_frame_b200/csrc/gdn_common.cuh",
+                  "hybrid_linear_attention_frame_b200/csrc/gdn_sm100.cuh"]
 
 
 def parse_args(argv=None):
@@ -53,7 +55,10 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target wall time of the oracle sample")
     ap.add_argument("--profile-tokens", type=int, default=0,
-                    help="profiling case: two gdn_forward calls on the layer's first T tokens, no timing")
+                    help="profiling case: two layer calls on the layer's first T tokens, no timing")
+    ap.add_argument("--path", choices=["ws", "plain"], default="ws",
+                    help="ws: gdn_forward_ws (shared prep through a workspace ring); "
+                         "plain: gdn_forward (no workspace)")
     return ap.parse_args(argv)
 
 
@@ -323,11 +328,17 @@ def run_ours(args, w, rank, world, local):
     dims = (w.B, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.chunk_len)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), b.data_ptr(), None,
             st_out.data_ptr(), out.data_ptr())
+    use_ws = args.path == "ws" and G.gdn_workspace_bytes(*dims[:5], w.chunk_len) > 0
+    ws = G.workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.chunk_len, device) if use_ws else None
+    ws_args = (ws.data_ptr(), ws.numel()) if use_ws else (None, 0)
 
     def layer_call():
-        st = lib.gdn_forward(*ptrs, *dims, sptr)
+        if use_ws:
+            st = lib.gdn_forward_ws(*ptrs, *dims, *ws_args, sptr)
+        else:
+            st = lib.gdn_forward(*ptrs, *dims, sptr)
         if st != 0:
-            raise G.GdnError(st, "gdn_forward")
+            raise G.GdnError(st, "gdn_forward_ws" if use_ws else "gdn_forward")
 
     for _ in range(args.warmup):
         for _ in range(layers):
@@ -373,7 +384,10 @@ def run_ours(args, w, rank, world, local):
     achieved = abytes / avg_launch_s / 1e9
     traffic, traffic_kernel = recorded_traffic()
     path = G.gdn_bf16_path(w.d_k, w.d_v, w.chunk_len)
-    kernel = "gdn_chunk_tc_kernel" if path == 1 else "chunk_ffma_kernel<bf16,64>"
+    if use_ws:
+        kernel = "gdn_ring_kernel"
+    else:
+        kernel = "gdn_chunk_tc_kernel" if path == 1 else "chunk_ffma_kernel<bf16,64>"
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": traffic if traffic_kernel == kernel else None,
@@ -390,7 +404,7 @@ def run_ours(args, w, rank, world, local):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(lib, G, w, device, stream, (h_q, h_k, h_v, h_g, h_b),
-                      (q, k, v, g, b), out, st_out, world, max(2, min(args.steps, 3)))
+                      (q, k, v, g, b), out, st_out, world, max(2, min(args.steps, 3)), ws)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -399,7 +413,12 @@ def run_ours(args, w, rank, world, local):
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": workload_config(w, layers), "roofline": roofline,
+            "data": "synthetic",
+            "config": dict(workload_config(w, layers),
+                           api=("gdn_forward_ws (C ABI, device buffers, workspace "
+                                f"{ws.numel() / 2**20:.1f} MiB reused by every layer)") if use_ws
+                           else "gdn_forward (C ABI, device buffers)"),
+            "roofline": roofline,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * layers,
             "clocks": clock_rec}
     if world > 1:
@@ -409,9 +428,9 @@ def run_ours(args, w, rank, world, local):
     return line if rank == 0 else None
 
 
-def run_e2e(lib, G, w, device, stream, host_src, dev, out, st_out, world, steps):
-    """The same metric through gdn_forward_host: pinned host inputs copied in,
-    output and final state copied out, every step."""
+def run_e2e(lib, G, w, device, stream, host_src, dev, out, st_out, world, steps, ws=None):
+    """The same metric through gdn_forward_host(_ws): pinned host inputs copied
+    in, output and final state copied out, every step."""
     import torch
     hq, hk, hv, hg, hb = (x.pin_memory() for x in host_src)
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -419,14 +438,19 @@ def run_e2e(lib, G, w, device, stream, host_src, dev, out, st_out, world, steps)
     q, k, v, g, b = dev
     sptr = stream.cuda_stream
 
+    host_args = (hq.data_ptr(), hk.data_ptr(), hv.data_ptr(), hg.data_ptr(), hb.data_ptr(), None,
+                 h_st.data_ptr(), h_out.data_ptr(), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                 g.data_ptr(), b.data_ptr(), st_out.data_ptr(), out.data_ptr(),
+                 w.B, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.chunk_len)
+    api = "gdn_forward_host_ws" if ws is not None else "gdn_forward_host"
+
     def call():
-        st = lib.gdn_forward_host(hq.data_ptr(), hk.data_ptr(), hv.data_ptr(), hg.data_ptr(),
-                                  hb.data_ptr(), None, h_st.data_ptr(), h_out.data_ptr(),
-                                  q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(),
-                                  b.data_ptr(), st_out.data_ptr(), out.data_ptr(),
-                                  w.B, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.chunk_len, sptr)
+        if ws is not None:
+            st = lib.gdn_forward_host_ws(*host_args, ws.data_ptr(), ws.numel(), sptr)
+        else:
+            st = lib.gdn_forward_host(*host_args, sptr)
         if st != 0:
-            raise G.GdnError(st, "gdn_forward_host")
+            raise G.GdnError(st, api)
 
     call()
     barrier(world, device)
@@ -442,11 +466,11 @@ def run_e2e(lib, G, w, device, stream, host_src, dev, out, st_out, world, steps)
     d2h = h_out.numel() * h_out.element_size() + h_st.numel() * 4
     return {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps,
-            "api": "gdn_forward_host (C ABI, pinned host buffers, one layer per step)"}
+            "api": f"{api} (C ABI, pinned host buffers, one layer per step)"}
 
 
-def run_profile_case(w, tokens):
-    """Two gdn_forward calls (warm-up + the one a profiler captures) on the first
+def run_profile_case(w, tokens, path="ws"):
+    """Two layer calls (warm-up + the one a profiler captures) on the first
     `tokens` tokens of the layer; small enough for a many-pass ncu capture."""
     import numpy as np
     import torch
@@ -460,9 +484,14 @@ def run_profile_case(w, tokens):
     b = torch.from_numpy(inp.beta).cuda()
     out = torch.empty_like(v)
     st = torch.empty((w.B, w.H, w.d_k, w.d_v), dtype=torch.float32, device="cuda")
+    ws = G.workspace(w.B, w.H, tokens, w.d_k, w.d_v, w.chunk_len) if path == "ws" else None
     for _ in range(2):
-        G.gdn_forward(q, k, v, g, b, None, st, out, w.B, w.H, tokens, w.d_k, w.d_v, w.frame_len,
-                      w.chunk_len)
+        if ws is not None:
+            G.gdn_forward_ws(q, k, v, g, b, None, st, out, w.B, w.H, tokens, w.d_k, w.d_v,
+                             w.frame_len, w.chunk_len, ws)
+        else:
+            G.gdn_forward(q, k, v, g, b, None, st, out, w.B, w.H, tokens, w.d_k, w.d_v,
+                          w.frame_len, w.chunk_len)
     torch.cuda.synchronize()
     status = G.gdn_get_last_device_status()
     print(f"profile case: T={tokens}, device status {status}")
@@ -475,7 +504,7 @@ def main(argv=None):
     from workloads import MINUTE
     w = MINUTE
     if args.profile_tokens > 0:
-        return run_profile_case(w, args.profile_tokens)
+        return run_profile_case(w, args.profile_tokens, args.path)
     if args.impl == "reference":
         line = run_reference(args, w, rank, world)
     else:

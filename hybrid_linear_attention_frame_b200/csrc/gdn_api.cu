@@ -13,6 +13,10 @@ template <typename IOT>
 cudaError_t launch_ffma(const FwdParams& p, int chunk_len, cudaStream_t stream);
 bool tc_supported(int dk, int dv, int chunk_len);
 cudaError_t launch_tc(const FwdParams& p, int chunk_len, cudaStream_t stream);
+bool ring_supported(int dk, int dv, int chunk_len);
+cudaError_t ring_groups(int BH, int dv, int* groups);
+size_t ring_workspace_bytes(int G, int dv);
+cudaError_t launch_ring(const FwdParams& p, void* ws, size_t ws_bytes, cudaStream_t stream);
 int read_and_clear_device_status(cudaStream_t stream);
 }  // namespace gdn
 
@@ -84,6 +88,78 @@ int run_bf16(const gdn::FwdParams& p, int chunk_len, cudaStream_t stream)
     return to_status(gdn::launch_ffma<__nv_bfloat16>(p, chunk_len, stream));
 }
 
+// Does this call take the shared-prep ring kernel (and so need a workspace)?
+bool uses_ring(int T, int dk, int dv, int chunk_len) { return T > 0 && gdn::ring_supported(dk, dv, chunk_len); }
+
+int workspace_need(int B, int H, int dv, size_t* need)
+{
+    int G = 0;
+    if (gdn::ring_groups(B * H, dv, &G) != cudaSuccess) return GDN_ERR_CUDA;
+    *need = gdn::ring_workspace_bytes(G, dv);
+    return GDN_OK;
+}
+
+// bf16 forward with a caller-provided workspace: the ring kernel where it
+// applies, else the workspace is not touched and the plain path runs.
+int run_bf16_ws(const gdn::FwdParams& p, int chunk_len, void* ws, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!uses_ring(p.T, p.dk, p.dv, chunk_len)) return run_bf16(p, chunk_len, stream);
+    size_t need = 0;
+    const int st = workspace_need(p.B, p.H, p.dv, &need);
+    if (st != GDN_OK) return st;
+    if (!ws || !aligned(ws, 256) || ws_bytes < need) return GDN_ERR_INVALID_ARG;
+    const int64_t F = ((int64_t)p.T + p.frame_len - 1) / p.frame_len;
+    const size_t nq = (size_t)p.B * p.T * p.H * p.dk * 2;
+    const size_t nv = (size_t)p.B * p.T * p.H * p.dv * 2;
+    const size_t ng = (size_t)p.B * F * p.H * sizeof(float);
+    const size_t nb = (size_t)p.B * p.T * p.H * sizeof(float);
+    const size_t ns = (size_t)p.B * p.H * p.dk * p.dv * sizeof(float);
+    if (overlaps(ws, need, p.q, nq) || overlaps(ws, need, p.k, nq) || overlaps(ws, need, p.v, nv) ||
+        overlaps(ws, need, p.gate, ng) || overlaps(ws, need, p.beta, nb) ||
+        overlaps(ws, need, p.state_in, ns) || overlaps(ws, need, p.state_out, ns) ||
+        overlaps(ws, need, p.out, nv))
+        return GDN_ERR_INVALID_ARG;
+    return to_status(gdn::launch_ring(p, ws, ws_bytes, stream));
+}
+
+int forward_host(const void* h_q, const void* h_k, const void* h_v,
+                     const float* h_gate_logit, const float* h_beta_logit,
+                     const float* h_state_in, float* h_state_out, void* h_out,
+                     void* d_q, void* d_k, void* d_v,
+                     float* d_gate_logit, float* d_beta_logit,
+                     float* d_state, void* d_out,
+                     int B, int H, int T, int d_k_dim, int d_v_dim,
+                     int frame_len, int chunk_len, void* ws, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!h_q || !h_k || !h_v || !h_gate_logit || !h_beta_logit || !h_out) return GDN_ERR_INVALID_ARG;
+    if ((h_state_in || h_state_out) && !d_state) return GDN_ERR_INVALID_ARG;
+    gdn::FwdParams p;
+    int st = validate(d_q, d_k, d_v, d_gate_logit, d_beta_logit, h_state_in ? d_state : nullptr,
+                      d_state, d_out, true, 2, B, H, T, d_k_dim, d_v_dim, frame_len,
+                      chunk_len, &p);
+    if (st != GDN_OK) return st;
+    const int64_t F = ((int64_t)T + frame_len - 1) / frame_len;
+    const size_t nq = (size_t)B * T * H * d_k_dim * 2;
+    const size_t nv = (size_t)B * T * H * d_v_dim * 2;
+    const size_t ng = (size_t)B * F * H * sizeof(float);
+    const size_t nb = (size_t)B * T * H * sizeof(float);
+    const size_t ns = (size_t)B * H * d_k_dim * d_v_dim * sizeof(float);
+    cudaError_t e = cudaSuccess;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_q, h_q, nq, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_k, h_k, nq, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_v, h_v, nv, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_gate_logit, h_gate_logit, ng, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d_beta_logit, h_beta_logit, nb, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess && h_state_in) e = cudaMemcpyAsync(d_state, h_state_in, ns, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    st = run_bf16_ws(p, chunk_len, ws, ws_bytes, stream);
+    if (st != GDN_OK) return st;
+    e = cudaMemcpyAsync(h_out, d_out, nv, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess && h_state_out) e = cudaMemcpyAsync(h_state_out, d_state, ns, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    return to_status(e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -151,33 +227,65 @@ int gdn_forward_host(const void* h_q, const void* h_k, const void* h_v,
                      int B, int H, int T, int d_k_dim, int d_v_dim,
                      int frame_len, int chunk_len, cudaStream_t stream)
 {
-    if (!h_q || !h_k || !h_v || !h_gate_logit || !h_beta_logit || !h_out) return GDN_ERR_INVALID_ARG;
-    if ((h_state_in || h_state_out) && !d_state) return GDN_ERR_INVALID_ARG;
+    return forward_host(h_q, h_k, h_v, h_gate_logit, h_beta_logit, h_state_in, h_state_out, h_out, d_q, d_k,
+                        d_v, d_gate_logit, d_beta_logit, d_state, d_out, B, H, T, d_k_dim, d_v_dim, frame_len,
+                        chunk_len, nullptr, 0, stream);
+}
+
+int gdn_forward_host_ws(const void* h_q, const void* h_k, const void* h_v,
+                        const float* h_gate_logit, const float* h_beta_logit,
+                        const float* h_state_in, float* h_state_out, void* h_out,
+                        void* d_q, void* d_k, void* d_v,
+                        float* d_gate_logit, float* d_beta_logit,
+                        float* d_state, void* d_out,
+                        int B, int H, int T, int d_k_dim, int d_v_dim,
+                        int frame_len, int chunk_len, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream)
+{
+    if (uses_ring(T, d_k_dim, d_v_dim, chunk_len) && !workspace) return GDN_ERR_INVALID_ARG;
+    return forward_host(h_q, h_k, h_v, h_gate_logit, h_beta_logit, h_state_in, h_state_out, h_out, d_q, d_k,
+                        d_v, d_gate_logit, d_beta_logit, d_state, d_out, B, H, T, d_k_dim, d_v_dim, frame_len,
+                        chunk_len, workspace, workspace_bytes, stream);
+}
+
+int gdn_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk_len, size_t* bytes)
+{
+    if (!bytes) return GDN_ERR_INVALID_ARG;
+    *bytes = 0;
+    if (B < 1 || H < 1 || T < 0 || (int64_t)B * H > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (!supported_dim(d_k) || !supported_dim(d_v)) return GDN_ERR_UNSUPPORTED;
+    if (chunk_len != 16 && chunk_len != 32 && chunk_len != 64) return GDN_ERR_UNSUPPORTED;
+    if (!uses_ring(T, d_k, d_v, chunk_len)) return GDN_OK;
+    return workspace_need(B, H, d_v, bytes);
+}
+
+int gdn_forward_ws(const void* q, const void* k, const void* v,
+                   const float* gate_logit, const float* beta_logit,
+                   const float* state_in, float* state_out, void* out,
+                   int B, int H, int T, int d_k, int d_v,
+                   int frame_len, int chunk_len, void* workspace, size_t workspace_bytes,
+                   cudaStream_t stream)
+{
     gdn::FwdParams p;
-    int st = validate(d_q, d_k, d_v, d_gate_logit, d_beta_logit, h_state_in ? d_state : nullptr,
-                      d_state, d_out, true, 2, B, H, T, d_k_dim, d_v_dim, frame_len,
-                      chunk_len, &p);
+    int st = validate(q, k, v, gate_logit, beta_logit, state_in, state_out, out, true, 2,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
     if (st != GDN_OK) return st;
-    const int64_t F = ((int64_t)T + frame_len - 1) / frame_len;
-    const size_t nq = (size_t)B * T * H * d_k_dim * 2;
-    const size_t nv = (size_t)B * T * H * d_v_dim * 2;
-    const size_t ng = (size_t)B * F * H * sizeof(float);
-    const size_t nb = (size_t)B * T * H * sizeof(float);
-    const size_t ns = (size_t)B * H * d_k_dim * d_v_dim * sizeof(float);
-    cudaError_t e = cudaSuccess;
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d_q, h_q, nq, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d_k, h_k, nq, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d_v, h_v, nv, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d_gate_logit, h_gate_logit, ng, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d_beta_logit, h_beta_logit, nb, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess && h_state_in) e = cudaMemcpyAsync(d_state, h_state_in, ns, cudaMemcpyHostToDevice, stream);
-    if (e != cudaSuccess) return GDN_ERR_CUDA;
-    st = run_bf16(p, chunk_len, stream);
+    return run_bf16_ws(p, chunk_len, workspace, workspace_bytes, stream);
+}
+
+int gdn_state_step_ws(const void* q, const void* k, const void* v,
+                      const float* gate_logit, const float* beta_logit,
+                      float* state, void* out,
+                      int B, int H, int T, int d_k, int d_v,
+                      int frame_len, int chunk_len, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream)
+{
+    if (!state) return GDN_ERR_INVALID_ARG;
+    gdn::FwdParams p;
+    int st = validate(q, k, v, gate_logit, beta_logit, state, state, out, false, 2,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
     if (st != GDN_OK) return st;
-    e = cudaMemcpyAsync(h_out, d_out, nv, cudaMemcpyDeviceToHost, stream);
-    if (e == cudaSuccess && h_state_out) e = cudaMemcpyAsync(h_state_out, d_state, ns, cudaMemcpyDeviceToHost, stream);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-    return to_status(e);
+    return run_bf16_ws(p, chunk_len, workspace, workspace_bytes, stream);
 }
 
 const char* gdn_status_string(int status)

@@ -2,4 +2,5 @@
 #include "gdn_status.cu"
 #include "gdn_ffma.cu"
 #include "gdn_tc.cu"
+#include "gdn_ring.cu"
 #include "gdn_api.cu"

@@ -1,0 +1,859 @@
+// Tensor-core chunked GDN forward for sm_100a with the state-independent work
+// of every chunk done ONCE per head and shared through an L2-resident ring.
+//
+// A head's d_k x d_v state is split into d_v / 16 column blocks, one CTA each
+// (a "group" of CTAs per head).  The per-chunk work splits in two halves
+// (notation of gdn_common.cuh):
+//
+//   prep  (depends on the chunk's inputs only)
+//     gates, [K;Q][K;Q]^T on the tensor cores, norms, A and P with the decay,
+//     T = (I+A)^{-1} diag(beta) (CUDA cores + mma.sync), W = T diag(e^G/|k|) K
+//     and U = T V for all d_v columns (tensor cores)
+//   chain (depends on the state; sequential over chunks)
+//     [Q;W] S, E = U - W S, K^T diag(e^{G_L-G}/|k|) E and P E, the state update
+//     and the output O = diag(e^G/|q|) Q S + P E.
+//
+// Prep of chunk n is done by CTA n mod (d_v/16) of the group, which writes the
+// chunk's record (W and P as ready-made 128-byte-swizzled operand images, U in
+// 16-column slices, the per-token scalars) into ring slot n mod kRing and then
+// publishes it with a GPU-scope release store.  Every CTA of the group runs the
+// chain for its own 16 columns over all chunks: a loader warp acquires the
+// record, pulls it into shared memory with bulk copies (plus the chunk's q and
+// k tiles by TMA) and reports the slot consumed once the copies have landed.
+// A producer re-fills a slot only after every CTA of the group has consumed
+// it.  Each wait depends only on chunks with a smaller index, and the launch is
+// cooperative (all CTAs resident), so the protocol cannot deadlock; every wait
+// is bounded all the same and gives up with GDN_ERR_TIMEOUT.
+//
+// Groups are persistent: group g serves chains g, g + G, g + 2G, ... back to
+// back, numbering their chunks consecutively.
+//
+// Warp roles inside a CTA: warps 0-3 run the chain, warps 4-11 the prep of
+// this CTA's share of the chunks, warp 12 loads the chain's records.
+#include <cudaTypedefs.h>
+
+#include "gdn_common.cuh"
+#include "gdn_status.cuh"
+#include "gdn_sm100.cuh"
+
+namespace gdn {
+namespace ring {
+
+using namespace sm100;
+using tc::kC;
+using tc::kXS;
+
+constexpr int kVB = 16;                // state columns per CTA
+constexpr int kThreads = 416;          // 13 warps
+constexpr int kChainThreads = 128;     // warps 0-3
+constexpr int kPrepThreads = 256;      // warps 4-11
+constexpr int kLoaderWarp = 12;
+constexpr uint32_t kBarChain = 1, kBarPrep = 2;   // named barriers (3 is the inverse's)
+constexpr int kRing = 16;              // record slots per group
+constexpr uint32_t kTmemCols = 512;
+
+// TMEM columns
+constexpr uint32_t kColG = 0;          // [K;Q][K;Q]^T     128 (prep)
+constexpr uint32_t kColW = 128;        // [T';T] K         128 (prep; lanes 0-63 = W)
+constexpr uint32_t kColU = 256;        // [T';T] V         128 (prep; lanes 64-127 = U)
+constexpr uint32_t kColQW = 384;       // [Q;W] S          16  (chain)
+constexpr uint32_t kColS = 400;        // K^T E'           16  (chain)
+constexpr uint32_t kColPE = 416;       // [P;X] E          2 x 16 (chain)
+
+// ---- record (global memory, one per ring slot) ----
+constexpr uint32_t kRecW = 0;          // W image: d-columns 0-63 | 64-127, 8 KB each (SW128)
+constexpr uint32_t kRecP = 16384;      // P image, 8 KB (SW128)
+constexpr uint32_t kRecU = 24576;      // U: per 16-column block [4][64][4] fp32 (4 KB)
+__host__ __device__ constexpr uint32_t rec_sc(int dv) { return kRecU + (uint32_t)(dv / 16) * 4096u; }
+__host__ __device__ constexpr uint32_t rec_bytes(int dv) { return rec_sc(dv) + 1024u; }
+constexpr uint32_t kScCopy = 528;      // GQ[64], DL[64], e^{G_L}, padding
+enum : uint32_t { RS_GQ = 0, RS_DL = 64, RS_GL = 128 };
+
+// ---- flags (start of the workspace) ----
+// word 0: abort; then per group: ready[kRing], consumed[8] (uint64 each)
+constexpr uint32_t kGroupFlags = kRing + 8;
+__host__ __device__ constexpr size_t flags_bytes(int G) {
+    return ((size_t)(1 + G * kGroupFlags) * 8 + 4095) / 4096 * 4096;
+}
+
+// ---- shared memory (from a 1024-aligned base) ----
+// chain slot: Q0 | W0 | Q1 | W1 | K0 | K1 | P | U | scalars
+constexpr uint32_t kTile = 8192;
+constexpr uint32_t cQ0 = 0, cW0 = 8192, cQ1 = 16384, cW1 = 24576, cK0 = 32768, cK1 = 40960;
+constexpr uint32_t cP = 49152, cU = 57344, cSc = 61440;
+constexpr uint32_t kCSlot = 62464;
+constexpr uint32_t kCHalfQ = cQ1 - cQ0;            // [Q;W] of d-columns 64-127
+constexpr uint32_t kCHalfK = cK1 - cK0;            // LBO of K^T (MN-major)
+// prep area: K0 | Q0 | K1 | Q1 | V0 | V1, then T' | T, AXI, scalars
+constexpr uint32_t kOffPrep = 2 * kCSlot;
+constexpr uint32_t pK0 = 0, pQ0 = 8192, pK1 = 16384, pQ1 = 24576, pV0 = 32768, pV1 = 40960;
+constexpr uint32_t kPHalf = pK1 - pK0;
+constexpr uint32_t kOffTp = kOffPrep + 49152;
+constexpr uint32_t kOffT = kOffTp + kTile;
+constexpr uint32_t kOffAXI = kOffT + kTile;
+constexpr uint32_t kScFloats = 13 * 64 + 16;
+constexpr uint32_t kOffSc = kOffAXI + 64 * kXS * 4;
+constexpr uint32_t kOffSB = ((kOffSc + kScFloats * 4 + 255) / 256) * 256;   // S bf16, SW32
+constexpr uint32_t kOffEB = kOffSB + 128 * 32;     // E  bf16, SW32
+constexpr uint32_t kOffEP = kOffEB + 64 * 32;      // E' bf16, SW32
+constexpr uint32_t kOffBar = kOffEP + 64 * 32;
+// barriers: full[2], cfree[2] (chain ring), ptma, g1, wu (prep), m1, m2 (chain)
+constexpr uint32_t kBarFull = 0, kBarFree = 2, kBarPTma = 4, kBarG1 = 5, kBarWU = 6, kBarM1 = 7,
+                   kBarM2 = 8, kNumBars = 9;
+constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+constexpr uint32_t kSmemUsed = kOffAbort + 4;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;
+
+// prep scalar table (floats)
+enum : uint32_t {
+    SC_G = 0, SC_BETA = 64, SC_RK = 128, SC_RQ = 192, SC_GQ = 256, SC_GAM = 320, SC_DL = 384,
+    SC_EXR = 448, SC_EXC = 512, SC_BGK = 768, SC_MISC = 832,
+};
+
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kCSlot % 1024 == 0 && kOffPrep % 1024 == 0 && kOffTp % 1024 == 0, "SW128 alignment");
+static_assert(4 * tc::kMS * 32 * 4 <= kTile, "solve scratch fits in the T tile");
+// P E reads a 128-row A operand from P; rows 64-127 (never read back) must stay in shared memory
+static_assert(kCSlot + cP + 2 * kTile <= kSmemUsed, "P operand over-read stays inside the allocation");
+
+constexpr uint32_t kIdG1 = idesc_bf16(128, 128, false, false);
+constexpr uint32_t kIdM1 = idesc_bf16(128, 16, false, true);
+constexpr uint32_t kIdM2S = idesc_bf16(128, 16, true, true);
+constexpr uint32_t kIdM2P = idesc_bf16(128, 16, false, true);
+
+struct RingArgs {
+    FwdParams p;
+    uint8_t* ws;             // workspace: flags, then G * kRing records
+    int G;                   // groups (persistent)
+    int ncb;                 // CTAs per group = d_v / 16
+    uint64_t wait_limit_ns;
+};
+
+__device__ __forceinline__ uint64_t kmaj128(uint32_t addr) { return smem_desc(addr, 16, 1024, kSwizzle128); }
+__device__ __forceinline__ uint64_t mnmaj128(uint32_t addr, uint32_t lbo) { return smem_desc(addr, lbo, 1024, kSwizzle128); }
+__device__ __forceinline__ uint64_t mnmaj32(uint32_t addr) { return smem_desc(addr, 256, 256, kSwizzle32); }
+
+// K step `ks` (16 elements) of a K-major operand whose d axis is split into two
+// SW128 column groups `half` bytes apart.
+__device__ __forceinline__ uint32_t dstep(uint32_t tile, int ks, uint32_t half) {
+    return tile + (ks >= 4 ? half : 0u) + (uint32_t)(ks & 3) * 32u;
+}
+
+__device__ __forceinline__ uint32_t tmem_lane(uint32_t tmem, int quarter) {
+    return tmem + ((uint32_t)(32 * quarter) << 16);
+}
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+__device__ __forceinline__ float softplus_fast(float x) {
+    return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x)));
+}
+__device__ __forceinline__ float sigmoid_fast(float x) {
+    return __fdividef(1.0f, 1.0f + __expf(-x));
+}
+
+// Group-local barrier that also returns the AND of `v` over the group.
+__device__ __forceinline__ bool group_all(uint32_t id, uint32_t n, bool v) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.u32 p, %3, 0;\n\t"
+                 "bar.red.and.pred q, %1, %2, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"(id), "r"(n), "r"(v ? 1u : 0u) : "memory");
+    return r != 0;
+}
+
+// Row `row` of a 16-column bf16 tile in the SW32 layout.
+__device__ __forceinline__ void store_row16_sw32(uint32_t tile, uint32_t row, const float (&x)[16]) {
+    st_shared_v4(tile + sw32_chunk_offset(row, 0), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                 pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+    st_shared_v4(tile + sw32_chunk_offset(row, 1), pack_bf16x2(x[8], x[9]), pack_bf16x2(x[10], x[11]),
+                 pack_bf16x2(x[12], x[13]), pack_bf16x2(x[14], x[15]));
+}
+
+__device__ __forceinline__ void store8_sw128(uint32_t tile, uint32_t row, uint32_t col, const float* x) {
+    st_shared_v4(tile + sw128_offset(row, col), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                 pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+}
+
+// 8 consecutive columns of row `row` of a SW128 image in global memory.
+__device__ __forceinline__ void gstore8_sw128(uint8_t* img, uint32_t row, uint32_t col, const float* x) {
+    st_global_v4(img + sw128_offset(row, col), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                 pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+}
+
+// Spin (bounded) until *flag >= want.  Gives up, raising both abort words and
+// recording `code`, after `limit_ns` or as soon as an abort word is raised.
+__device__ __forceinline__ bool wait_flag(const uint64_t* flag, uint64_t want, volatile int* abort_cta,
+                                          uint64_t* abort_glob, uint64_t limit_ns, int code) {
+    if (ld_acquire_u64(flag) >= want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(32);
+        if (ld_acquire_u64(flag) >= want) return true;
+        if ((it & 15u) == 0) {
+            if (*abort_cta || *reinterpret_cast<volatile uint64_t*>(abort_glob) != 0) {
+                *abort_cta = 1;
+                return false;
+            }
+            if (globaltimer_ns() - t0 > limit_ns) {
+                *abort_cta = 1;
+                *reinterpret_cast<volatile uint64_t*>(abort_glob) = 1;
+                atomicCAS(&g_device_status, 0, code);
+                return false;
+            }
+        }
+    }
+}
+
+// Where chunk n of group g lives: chain index and chunk within the chain.
+struct Item {
+    int b, h, c, L;
+};
+__device__ __forceinline__ Item item_of(const FwdParams& p, int g, int G, int ntk, int n) {
+    Item it;
+    const int x = g + (n / ntk) * G;
+    it.b = x / p.H;
+    it.h = x % p.H;
+    it.c = n % ntk;
+    it.L = min(kC, p.T - it.c * kC);
+    return it;
+}
+
+
+// Bounded wait used only on the way out after an abort (async copies or MMAs
+// that may still be in flight must land before shared memory and TMEM go).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < limit_ns) {
+    }
+}
+
+// ---------------------------------------------------------------- MMA issue (one warp)
+
+// prep: [K;Q][K;Q]^T (M = N = 128, K = d_k)
+__device__ __forceinline__ void issue_g1(uint32_t prep, uint32_t tmem, int nks) {
+    for (int ks = 0; ks < nks; ++ks) {
+        const uint64_t a = kmaj128(dstep(prep + pK0, ks, kPHalf));
+        mma_bf16_warp(tmem + kColG, a, a, kIdG1, ks > 0);
+    }
+}
+
+// prep: [T';T] K (N = d_k) and [T';T] V (N = d_v), K = 64 tokens
+__device__ __forceinline__ void issue_wu(uint32_t prep, uint32_t tp, uint32_t tmem, int dk, int dv) {
+    const uint32_t idw = idesc_bf16(128, dk, false, true);
+    const uint32_t idu = idesc_bf16(128, dv, false, true);
+#pragma unroll
+    for (int ks = 0; ks < kC / 16; ++ks) {
+        const uint64_t a = kmaj128(tp + (uint32_t)ks * 32u);
+        mma_bf16_warp(tmem + kColW, a, mnmaj128(prep + pK0 + (uint32_t)ks * 2048u, kPHalf), idw, ks > 0);
+        mma_bf16_warp(tmem + kColU, a, mnmaj128(prep + pV0 + (uint32_t)ks * 2048u, pV1 - pV0), idu, ks > 0);
+    }
+}
+
+// chain: [Q;W] S (M = 128, N = 16, K = d_k)
+__device__ __forceinline__ void issue_m1(uint32_t slot, uint32_t sb, uint32_t tmem, int nks) {
+    for (int ks = 0; ks < nks; ++ks)
+        mma_bf16_warp(tmem + kColQW, kmaj128(dstep(slot + cQ0, ks, kCHalfQ)), mnmaj32(sb + (uint32_t)ks * 512u),
+                      kIdM1, ks > 0);
+}
+
+// chain: K^T E' (M = 128 over d_k) and [P;X] E (rows 0-63 used), K = 64 tokens
+__device__ __forceinline__ void issue_m2(uint32_t slot, uint32_t eb, uint32_t ep, uint32_t tmem, int s) {
+#pragma unroll
+    for (int ks = 0; ks < kC / 16; ++ks) {
+        mma_bf16_warp(tmem + kColS, mnmaj128(slot + cK0 + (uint32_t)ks * 2048u, kCHalfK),
+                      mnmaj32(ep + (uint32_t)ks * 512u), kIdM2S, ks > 0);
+        mma_bf16_warp(tmem + kColPE + 16u * s, kmaj128(slot + cP + (uint32_t)ks * 32u),
+                      mnmaj32(eb + (uint32_t)ks * 512u), kIdM2P, ks > 0);
+    }
+}
+
+// ---------------------------------------------------------------- the kernel
+
+__global__ void __launch_bounds__(kThreads, 1)
+gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const RingArgs args)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gb = smem_raw + (base - raw);
+    const FwdParams& p = args.p;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, qtr = warp & 3;
+    const int vb = blockIdx.x, g = blockIdx.y, G = args.G, ncb = args.ncb;
+    const int dk = p.dk, dv = p.dv, nks = dk / 16;
+    const int ntk = (p.T + kC - 1) / kC;
+    const int nchains = (p.B * p.H - g + G - 1) / G;
+    const int total = nchains * ntk;                  // chunks served by this group
+    const uint32_t recb = rec_bytes(dv);
+    uint64_t* abort_glob = reinterpret_cast<uint64_t*>(args.ws);
+    uint64_t* ready = abort_glob + 1 + (size_t)g * kGroupFlags;
+    uint64_t* consumed = ready + kRing;
+    uint8_t* recs = args.ws + flags_bytes(G) + (size_t)g * kRing * recb;
+
+    float* AXI = reinterpret_cast<float*>(gb + kOffAXI);
+    float* MSf = reinterpret_cast<float*>(gb + kOffT);
+    float* sc = reinterpret_cast<float*>(gb + kOffSc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + kOffAbort);
+    const uint32_t bars = base + kOffBar;
+    auto bar = [&](uint32_t i) { return bars + 8u * i; };
+    const uint32_t sbt = base + kOffSB, ebt = base + kOffEB, ept = base + kOffEP;
+    const uint32_t prep = base + kOffPrep;
+    const uint64_t lim = args.wait_limit_ns;
+
+    if (warp == 0) {
+        tmem_alloc(base + kOffTmemSlot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 32) {
+        for (uint32_t i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+        fence_mbar_init();
+        *abort_flag = 0;
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gb + kOffTmemSlot);
+
+    if (warp < 4) {
+        // ======================= chain =======================
+        float S[16], QS[16];
+        float gq = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) { S[j] = 0.0f; QS[j] = 0.0f; }
+        bool ok = true, m1_pending = false, m2_pending = false;
+        int pend_n = -1;                      // item whose output is still to be written
+        Item pend{0, 0, 0, 0};
+        // O = diag(e^G/|q|) Q S + P E of item n (warps 0, 1; rows 32*qtr + lane)
+        auto output = [&](const Item& it, int n) {
+            if (qtr >= 2) return;
+            const int i = 32 * qtr + lane;
+            float pe[16];
+            tmem_ld16(tmem_lane(tmem, qtr) + kColPE + 16u * (uint32_t)(n & 1), pe);
+            tmem_wait_ld();
+            if (i < it.L && p.out) {
+                uint32_t w[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    w[j] = pack_bf16x2(fmaf(gq, QS[2 * j], pe[2 * j]), fmaf(gq, QS[2 * j + 1], pe[2 * j + 1]));
+                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) +
+                                   (((size_t)it.b * p.T + (size_t)it.c * kC + i) * p.H + it.h) * dv +
+                                   (size_t)vb * kVB;
+                uint4* o4 = reinterpret_cast<uint4*>(o);
+                o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+        };
+        for (int n = 0; n < total; ++n) {
+            const Item it = item_of(p, g, G, ntk, n);
+            const int s = n & 1;
+            const uint32_t slot = base + (uint32_t)s * kCSlot;
+            const float* csc = reinterpret_cast<const float*>(gb + (uint32_t)s * kCSlot + cSc);
+            const float* cu = reinterpret_cast<const float*>(gb + (uint32_t)s * kCSlot + cU);
+            if (it.c == 0) {
+                // first chunk of a chain: its initial state (this thread owns row tid)
+                const size_t sbase = ((size_t)it.b * p.H + it.h) * (size_t)dk * dv + (size_t)vb * kVB;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) S[j] = 0.0f;
+                if (p.state_in && tid < dk) {
+                    const float4* si = reinterpret_cast<const float4*>(p.state_in + sbase + (size_t)tid * dv);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float4 v4 = si[j];
+                        S[4 * j] = v4.x; S[4 * j + 1] = v4.y; S[4 * j + 2] = v4.z; S[4 * j + 3] = v4.w;
+                    }
+                }
+                if (tid < dk) store_row16_sw32(sbt, (uint32_t)tid, S);
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(kBarChain, kChainThreads);
+            }
+            ok = mbar_wait(bar(kBarFull + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 11);
+            if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
+            if (tid == 0) {
+                // the record is in shared memory: its ring slot may be re-filled
+                fence_proxy_async_global();
+                st_release_u64(consumed + vb, (uint64_t)n + 1);
+            }
+            tc_fence_after();
+            if (warp == 0) {
+                issue_m1(slot, sbt, tmem, nks);
+                mma_commit_warp(bar(kBarM1));
+            }
+            m1_pending = true;
+            if (it.c > 0) output(pend, pend_n);        // previous chunk's output while MMA1 runs
+            ok = mbar_wait(bar(kBarM1), (uint32_t)(n & 1), abort_flag, lim, 4);
+            if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
+            m1_pending = false;
+            tc_fence_after();
+            {
+                float v[16];
+                tmem_ld16(tmem_lane(tmem, qtr) + kColQW, v);
+                if (qtr < 2) {
+                    gq = csc[RS_GQ + 32 * qtr + lane];
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) QS[j] = v[j];
+                } else {
+                    const int i = 32 * (qtr - 2) + lane;
+                    float u[16];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 u4 = ld4(cu + q * 256 + i * 4);
+                        u[4 * q] = u4.x; u[4 * q + 1] = u4.y; u[4 * q + 2] = u4.z; u[4 * q + 3] = u4.w;
+                    }
+                    const float d = csc[RS_DL + i];
+                    tmem_wait_ld();
+                    float e[16], e2[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        e[j] = u[j] - v[j];
+                        e2[j] = e[j] * d;
+                    }
+                    store_row16_sw32(ebt, (uint32_t)i, e);
+                    store_row16_sw32(ept, (uint32_t)i, e2);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(kBarChain, kChainThreads);
+            if (warp == 0) {
+                tc_fence_after();
+                issue_m2(slot, ebt, ept, tmem, s);
+                mma_commit_warp(bar(kBarM2));
+            }
+            m2_pending = true;
+            ok = mbar_wait(bar(kBarM2), (uint32_t)(n & 1), abort_flag, lim, 5);
+            if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
+            m2_pending = false;
+            tc_fence_after();
+            {
+                float v[16];
+                tmem_ld16(tmem_lane(tmem, qtr) + kColS, v);
+                const float gL = csc[RS_GL];
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) S[j] = fmaf(gL, S[j], v[j]);
+                if (tid < dk) store_row16_sw32(sbt, (uint32_t)tid, S);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(kBarChain, kChainThreads);
+            if (tid == 0) mbar_arrive(bar(kBarFree + s));   // slot s back to the loader
+            pend = it;
+            pend_n = n;
+            if (it.c == ntk - 1) {
+                // last chunk of the chain: its output and the final state
+                output(it, n);
+                if (p.state_out && tid < dk) {
+                    const size_t sbase = ((size_t)it.b * p.H + it.h) * (size_t)dk * dv + (size_t)vb * kVB;
+                    float4* so = reinterpret_cast<float4*>(p.state_out + sbase + (size_t)tid * dv);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        so[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+                }
+            }
+        }
+        if (!ok && (m1_pending || m2_pending)) {
+            // one parity is already complete, the other waits for the MMAs still in flight
+            const uint32_t mb = bar(m1_pending ? kBarM1 : kBarM2);
+            drain_wait(mb, 0, lim);
+            drain_wait(mb, 1, lim);
+        }
+    } else if (warp < 12) {
+        // ======================= prep =======================
+        const int pt = tid - kChainThreads;   // 0..255
+        const int pw = warp - 4;              // 0..7
+        bool ok = true;
+        int mma_pending = -1;                 // barrier of an MMA group not yet waited for
+        int ptma_issued = 0, ptma_waited = 0;
+        auto issue_prep_tma = [&](int nn) {
+            const Item jt = item_of(p, g, G, ntk, nn);
+            const uint32_t pb = bar(kBarPTma);
+            const int t0 = jt.c * kC;
+            mbar_arrive_expect_tx(pb, 6 * kTile);
+            tma_load_4d(prep + pK0, &tm_k, pb, 0, jt.h, t0, jt.b);
+            tma_load_4d(prep + pQ0, &tm_q, pb, 0, jt.h, t0, jt.b);
+            tma_load_4d(prep + pK1, &tm_k, pb, 64, jt.h, t0, jt.b);
+            tma_load_4d(prep + pQ1, &tm_q, pb, 64, jt.h, t0, jt.b);
+            tma_load_4d(prep + pV0, &tm_v, pb, 0, jt.h, t0, jt.b);
+            tma_load_4d(prep + pV1, &tm_v, pb, 64, jt.h, t0, jt.b);
+        };
+        if (vb < total) {
+            if (pw == 4 && elect_one()) issue_prep_tma(vb);
+            ptma_issued = 1;
+        }
+        int m = 0;
+        for (int n = vb; n < total; n += ncb, ++m) {
+            const Item it = item_of(p, g, G, ntk, n);
+            const int L = it.L;
+            uint8_t* rec = recs + (size_t)(n % kRing) * recb;
+            // ---- the ring slot must have been consumed by every CTA of the group ----
+            bool got = true;
+            if (pt == 0 && n >= kRing)
+                for (int v = 0; v < ncb && got; ++v)
+                    got = wait_flag(consumed + v, (uint64_t)(n - kRing + 1), abort_flag, abort_glob, lim, 14);
+            // ---- gates: G (cumulative log-gate), beta ----
+            if (pw == 0) {
+                const int i0 = 2 * lane, i1 = i0 + 1, t0 = it.c * kC + i0;
+                float g0 = 0.0f, g1 = 0.0f, r0 = 0.0f, r1 = 0.0f;
+                if (i0 < L) {
+                    g0 = __ldg(p.gate + ((size_t)it.b * p.F + t0 / p.frame_len) * p.H + it.h);
+                    r0 = __ldg(p.beta + ((size_t)it.b * p.T + t0) * p.H + it.h);
+                }
+                if (i1 < L) {
+                    g1 = __ldg(p.gate + ((size_t)it.b * p.F + (t0 + 1) / p.frame_len) * p.H + it.h);
+                    r1 = __ldg(p.beta + ((size_t)it.b * p.T + t0 + 1) * p.H + it.h);
+                }
+                const float la0 = (i0 < L) ? -softplus_fast(g0) : 0.0f;
+                const float la1 = (i1 < L) ? -softplus_fast(g1) : 0.0f;
+                float x = la0 + la1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                sc[SC_G + i0] = x - la1;
+                sc[SC_G + i1] = x;
+                sc[SC_BETA + i0] = (i0 < L) ? sigmoid_fast(r0) : 0.0f;
+                sc[SC_BETA + i1] = (i1 < L) ? sigmoid_fast(r1) : 0.0f;
+            }
+            if (!group_all(kBarPrep, kPrepThreads, got)) { ok = false; break; }
+            {
+                const float GL = sc[SC_G + L - 1];
+                if (pt < 64) {
+                    const int i = pt;
+                    const float Gi = sc[SC_G + i];
+                    sc[SC_GAM + i] = __expf(Gi);
+                    sc[SC_DL + i] = (i < L) ? __expf(GL - Gi) : 0.0f;     // times 1/|k_i| below
+                    sc[SC_EXR + i] = (i >= 16) ? __expf(Gi - sc[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
+                    if (i == 0) sc[SC_MISC] = __expf(GL);
+                } else {
+                    const int idx = pt - 64;                  // 0..191
+                    const int bi = 1 + idx / 64, j = idx & 63;
+                    sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? __expf(sc[SC_G + 16 * bi - 1] - sc[SC_G + j]) : 0.0f;
+                }
+            }
+            // ---- [K;Q][K;Q]^T ----
+            ok = mbar_wait(bar(kBarPTma), (uint32_t)(m & 1), abort_flag, lim, 1);
+            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            ptma_waited = m + 1;
+            if (pw == 4) {
+                tc_fence_after();
+                issue_g1(prep, tmem, nks);
+                mma_commit_warp(bar(kBarG1));
+            }
+            mma_pending = kBarG1;
+            ok = mbar_wait(bar(kBarG1), (uint32_t)(m & 1), abort_flag, lim, 2);
+            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            mma_pending = -1;
+            tc_fence_after();
+            const uint32_t tg = tmem + kColG;
+            // ---- norms from the Gram diagonal: |k_i|^2 (lanes 0-63), |q_i|^2 (lanes 64-127) ----
+            if (pw < 4) {
+                float v[32];
+                tmem_ld16(tmem_lane(tg, qtr) + 32u * qtr, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_ld16(tmem_lane(tg, qtr) + 32u * qtr + 16u, *reinterpret_cast<float(*)[16]>(&v[16]));
+                tmem_wait_ld();
+                float d = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) d = (j == lane) ? v[j] : d;
+                const float r = rsqrtf(d + kNormEps);
+                const int i = 32 * (qtr & 1) + lane;
+                if (qtr < 2) {
+                    sc[SC_RK + i] = r;
+                    sc[SC_DL + i] *= r;
+                    sc[SC_BGK + i] = sc[SC_BETA + i] * sc[SC_GAM + i] * r;
+                } else {
+                    sc[SC_RQ + i] = r;
+                    sc[SC_GQ + i] = r * sc[SC_GAM + i];
+                }
+            }
+            named_bar_sync(kBarPrep, kPrepThreads);
+            // ---- A (fp32, transposed into AXI) and P (bf16 image in the record) ----
+            if ((qtr & 1) == 0 && (pw >> 2) == 1) {
+                // rows 0-31 x columns 32-63 lie above the diagonal: A has nothing there, P is zero
+                if (qtr == 2) {
+                    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int g8 = 0; g8 < 4; ++g8) gstore8_sw128(rec + kRecP, (uint32_t)lane, (uint32_t)(32 + 8 * g8), z);
+                }
+            } else {
+                const int ch = pw >> 2;
+                const int i = 32 * (qtr & 1) + lane;
+                const int bi = i >> 4;
+                const float Gi = sc[SC_G + i], exr = sc[SC_EXR + i];
+                const float ri = (qtr < 2) ? sc[SC_BETA + i] * sc[SC_RK + i] : sc[SC_RQ + i];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int j0 = 32 * ch + 16 * hh;
+                    float v[16], gj[16], rkj[16], ex[16];
+                    tmem_ld16(tmem_lane(tg, qtr) + (uint32_t)j0, v);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 a = ld4(sc + SC_G + j0 + 4 * q4);
+                        const float4 r4 = ld4(sc + SC_RK + j0 + 4 * q4);
+                        const float4 e4 = ld4(sc + SC_EXC + 64 * bi + j0 + 4 * q4);
+                        gj[4 * q4] = a.x; gj[4 * q4 + 1] = a.y; gj[4 * q4 + 2] = a.z; gj[4 * q4 + 3] = a.w;
+                        rkj[4 * q4] = r4.x; rkj[4 * q4 + 1] = r4.y; rkj[4 * q4 + 2] = r4.z; rkj[4 * q4 + 3] = r4.w;
+                        ex[4 * q4] = e4.x; ex[4 * q4 + 1] = e4.y; ex[4 * q4 + 2] = e4.z; ex[4 * q4 + 3] = e4.w;
+                    }
+                    tmem_wait_ld();
+                    float val[16];
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int j = j0 + jj;
+                        const float dec = ((j >> 4) == bi) ? __expf(Gi - gj[jj]) : exr * ex[jj];
+                        const bool keep = (qtr < 2) ? (j < i) : (j <= i);
+                        val[jj] = keep ? ri * rkj[jj] * v[jj] * dec : 0.0f;
+                    }
+                    if (qtr < 2) {
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            if (j0 + jj < i) AXI[(j0 + jj) * kXS + i] = val[jj];
+                    } else {
+                        gstore8_sw128(rec + kRecP, (uint32_t)i, (uint32_t)j0, &val[0]);
+                        gstore8_sw128(rec + kRecP, (uint32_t)i, (uint32_t)j0 + 8, &val[8]);
+                    }
+                }
+            }
+            tc_fence_before();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            if (pw < 4) {
+                // ---- T = (I + A)^{-1} diag(beta), T' = T diag(e^G / |k|) ----
+                tc::unit_lower_inverse_64(AXI, MSf, pt);
+                const int i = pt >> 1, j0 = 32 * (pt & 1);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int jb = j0 + 16 * q;
+                    float tv[16], tpv[16];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 x4 = ld4(AXI + i * kXS + jb + 4 * q4);
+                        const float4 b4 = ld4(sc + SC_BETA + jb + 4 * q4);
+                        const float4 f4 = ld4(sc + SC_BGK + jb + 4 * q4);
+                        const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+                        const float bs[4] = {b4.x, b4.y, b4.z, b4.w};
+                        const float fs[4] = {f4.x, f4.y, f4.z, f4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float x = (jb + 4 * q4 + e <= i) ? xs[e] : 0.0f;
+                            tv[4 * q4 + e] = x * bs[e];
+                            tpv[4 * q4 + e] = x * fs[e];
+                        }
+                    }
+                    store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)jb, &tv[0]);
+                    store8_sw128(base + kOffT, (uint32_t)i, (uint32_t)jb + 8, &tv[8]);
+                    store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)jb, &tpv[0]);
+                    store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)jb + 8, &tpv[8]);
+                }
+            } else {
+                // ---- the chain's per-token scalars into the record ----
+                float* rs = reinterpret_cast<float*>(rec + rec_sc(dv));
+                const int j = pt - 128;
+                if (j < 64) {
+                    rs[RS_GQ + j] = sc[SC_GQ + j];
+                    rs[RS_DL + j] = sc[SC_DL + j];
+                } else if (j < 68) {
+                    rs[RS_GL + (j - 64)] = (j == 64) ? sc[SC_MISC] : 0.0f;
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            if (pw == 0) {
+                tc_fence_after();
+                issue_wu(prep, base + kOffTp, tmem, dk, dv);
+                mma_commit_warp(bar(kBarWU));
+            }
+            mma_pending = kBarWU;
+            ok = mbar_wait(bar(kBarWU), (uint32_t)(m & 1), abort_flag, lim, 3);
+            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            mma_pending = -1;
+            tc_fence_after();
+            // the prep tiles are free: fetch the next item's
+            if (pw == 4 && n + ncb < total) {
+                if (elect_one()) {
+                    fence_proxy_async_smem();
+                    issue_prep_tma(n + ncb);
+                }
+                __syncwarp();
+            }
+            if (n + ncb < total) ptma_issued = m + 2;
+            // ---- W (TMEM lanes 0-63) and U (lanes 64-127) into the record ----
+            {
+                const int half = pw >> 2;
+                if (qtr < 2) {
+                    const int i = 32 * qtr + lane;
+                    for (int cb = 64 * half; cb < 64 * half + 64 && cb < dk; cb += 16) {
+                        float v[16];
+                        tmem_ld16(tmem_lane(tmem, qtr) + kColW + (uint32_t)cb, v);
+                        tmem_wait_ld();
+                        uint8_t* img = rec + kRecW + (cb >= 64 ? kTile : 0u);
+                        gstore8_sw128(img, (uint32_t)i, (uint32_t)(cb & 63), &v[0]);
+                        gstore8_sw128(img, (uint32_t)i, (uint32_t)(cb & 63) + 8, &v[8]);
+                    }
+                } else {
+                    const int i = 32 * (qtr - 2) + lane;
+                    for (int cb = 64 * half; cb < 64 * half + 64 && cb < dv; cb += 16) {
+                        float v[16];
+                        tmem_ld16(tmem_lane(tmem, qtr) + kColU + (uint32_t)cb, v);
+                        tmem_wait_ld();
+                        uint8_t* dst = rec + kRecU + (uint32_t)(cb / 16) * 4096u + (uint32_t)i * 16u;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            st_global_v4(dst + q * 1024, __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                         __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+                    }
+                }
+            }
+            tc_fence_before();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            if (pt == 0) {
+                // publish: every write of the record happens-before the release, and
+                // is ordered before the consumers' bulk copies (async proxy)
+                __threadfence();
+                fence_proxy_async_global();
+                st_release_u64(ready + (n % kRing), (uint64_t)n + 1);
+            }
+        }
+        if (!ok) {
+            if (pw == 4) {
+                if (ptma_issued > ptma_waited) drain_wait(bar(kBarPTma), (uint32_t)((ptma_issued - 1) & 1), lim);
+                if (mma_pending >= 0) {
+                    drain_wait(bar((uint32_t)mma_pending), 0, lim);
+                    drain_wait(bar((uint32_t)mma_pending), 1, lim);
+                }
+            }
+        }
+    } else {
+        // ======================= record loader (warp 12) =======================
+        bool ok = true;
+        int issued = 0;
+        for (int n = 0; n < total; ++n) {
+            const int s = n & 1;
+            if (n >= 2) {
+                ok = mbar_wait(bar(kBarFree + s), (uint32_t)(((n >> 1) - 1) & 1), abort_flag, lim, 12);
+                if (!ok) break;
+            }
+            bool got = true;
+            if (lane == 0) got = wait_flag(ready + (n % kRing), (uint64_t)n + 1, abort_flag, abort_glob, lim, 13);
+            got = __shfl_sync(0xffffffffu, got, 0);
+            if (!got) { ok = false; break; }
+            if (lane == 0) {
+                fence_proxy_async_global();
+                const Item it = item_of(p, g, G, ntk, n);
+                const uint8_t* rec = recs + (size_t)(n % kRing) * recb;
+                const uint32_t slot = base + (uint32_t)s * kCSlot;
+                const uint32_t fb = bar(kBarFull + s);
+                const int t0 = it.c * kC;
+                mbar_arrive_expect_tx(fb, 3 * kTile + 4096u + kScCopy + 4 * kTile);
+                bulk_load(slot + cW0, rec + kRecW, kTile, fb);
+                bulk_load(slot + cW1, rec + kRecW + kTile, kTile, fb);
+                bulk_load(slot + cP, rec + kRecP, kTile, fb);
+                bulk_load(slot + cU, rec + kRecU + (uint32_t)vb * 4096u, 4096u, fb);
+                bulk_load(slot + cSc, rec + rec_sc(dv), kScCopy, fb);
+                tma_load_4d(slot + cQ0, &tm_q, fb, 0, it.h, t0, it.b);
+                tma_load_4d(slot + cQ1, &tm_q, fb, 64, it.h, t0, it.b);
+                tma_load_4d(slot + cK0, &tm_k, fb, 0, it.h, t0, it.b);
+                tma_load_4d(slot + cK1, &tm_k, fb, 64, it.h, t0, it.b);
+            }
+            __syncwarp();
+            issued = n + 1;
+        }
+        if (!ok && lane == 0) {
+            // copies still in flight must land before shared memory goes away
+            for (int n = max(0, issued - 2); n < issued; ++n)
+                drain_wait(bar(kBarFull + (n & 1)), (uint32_t)((n >> 1) & 1), lim);
+        }
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace ring
+
+// ---------------------------------------------------------------- host side
+
+bool ring_supported(int dk, int dv, int chunk_len)
+{
+    // d > 64 keeps both 64-column TMA boxes of q, k and v partly inside the tensor
+    return chunk_len == ring::kC && dk % 16 == 0 && dk > 64 && dk <= 128 && dv % 16 == 0 && dv > 64 &&
+           dv <= 128;
+}
+
+// Number of persistent groups (heads in flight) for B*H chains on the current
+// device: every CTA of the cooperative grid must be resident at once.
+cudaError_t ring_groups(int BH, int dv, int* groups)
+{
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(ring::gdn_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)ring::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ring::gdn_ring_kernel, ring::kThreads,
+                                                          ring::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int ncb = dv / ring::kVB;
+    const int cap = (sms * per_sm) / ncb;
+    *groups = BH < cap ? BH : cap;
+    return *groups >= 1 ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+size_t ring_workspace_bytes(int G, int dv)
+{
+    return ring::flags_bytes(G) + (size_t)G * ring::kRing * ring::rec_bytes(dv);
+}
+
+cudaError_t launch_ring(const FwdParams& p, void* ws, size_t ws_bytes, cudaStream_t stream)
+{
+    if (!ring_supported(p.dk, p.dv, ring::kC) || p.T < 1) return cudaErrorInvalidValue;
+    int G = 0;
+    cudaError_t e = ring_groups(p.B * p.H, p.dv, &G);
+    if (e != cudaSuccess) return e;
+    if (ws_bytes < ring_workspace_bytes(G, p.dv)) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, p.q, p.dk, p.H, p.T, p.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mk, p.k, p.dk, p.H, p.T, p.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mv, p.v, p.dv, p.H, p.T, p.B, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    // the flags start from zero on every call; the records need no clearing
+    e = cudaMemsetAsync(ws, 0, ring::flags_bytes(G), stream);
+    if (e != cudaSuccess) return e;
+    ring::RingArgs args;
+    args.p = p;
+    args.ws = static_cast<uint8_t*>(ws);
+    args.G = G;
+    args.ncb = p.dv / ring::kVB;
+    args.wait_limit_ns = g_wait_limit_ns;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)args.ncb, (unsigned)G);
+    cfg.blockDim = dim3(ring::kThreads);
+    cfg.dynamicSmemBytes = ring::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ring::gdn_ring_kernel, mq, mk, mv, args);
+}
+
+}  // namespace gdn

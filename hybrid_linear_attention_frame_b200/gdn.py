@@ -20,7 +20,8 @@ GDN_ERR_CUDA = -3
 GDN_ERR_TIMEOUT = -4
 
 EXPORTS = ("gdn_forward", "gdn_state_step", "gdn_forward_f32", "gdn_state_step_f32",
-           "gdn_forward_host", "gdn_status_string", "gdn_get_last_device_status",
+           "gdn_forward_host", "gdn_workspace_bytes", "gdn_forward_ws", "gdn_state_step_ws",
+           "gdn_forward_host_ws", "gdn_status_string", "gdn_get_last_device_status",
            "gdn_bf16_path", "gdn_version")
 
 
@@ -59,6 +60,15 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         f.restype = I
     lib.gdn_forward_host.argtypes = [P] * 15 + [I] * 7 + [P]
     lib.gdn_forward_host.restype = I
+    Z = ctypes.c_size_t
+    lib.gdn_workspace_bytes.argtypes = [I] * 6 + [ctypes.POINTER(Z)]
+    lib.gdn_workspace_bytes.restype = I
+    lib.gdn_forward_ws.argtypes = [P] * 8 + [I] * 7 + [P, Z, P]
+    lib.gdn_forward_ws.restype = I
+    lib.gdn_state_step_ws.argtypes = [P] * 7 + [I] * 7 + [P, Z, P]
+    lib.gdn_state_step_ws.restype = I
+    lib.gdn_forward_host_ws.argtypes = [P] * 15 + [I] * 7 + [P, Z, P]
+    lib.gdn_forward_host_ws.restype = I
     lib.gdn_status_string.argtypes = [I]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_get_last_device_status.argtypes = [P]
@@ -143,6 +153,52 @@ def gdn_forward_host(h_q, h_k, h_v, h_gate_logit, h_beta_logit, h_state_in, h_st
     return _check(st, "gdn_forward_host", check)
 
 
+def gdn_workspace_bytes(B, H, T, d_k, d_v, chunk_len) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().gdn_workspace_bytes(B, H, T, d_k, d_v, chunk_len, ctypes.byref(n))
+    _check(st, "gdn_workspace_bytes", True)
+    return int(n.value)
+
+
+def _nbytes(ws) -> int:
+    return 0 if ws is None else ws.numel() * ws.element_size()
+
+
+def gdn_forward_ws(q, k, v, gate_logit, beta_logit, state_in, state_out, out,
+                   B, H, T, d_k, d_v, frame_len, chunk_len, workspace, workspace_bytes=None,
+                   stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().gdn_forward_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logit), _ptr(beta_logit),
+                               _ptr(state_in), _ptr(state_out), _ptr(out),
+                               B, H, T, d_k, d_v, frame_len, chunk_len, _ptr(workspace), wb,
+                               _stream(stream))
+    return _check(st, "gdn_forward_ws", check)
+
+
+def gdn_state_step_ws(q, k, v, gate_logit, beta_logit, state, out,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, workspace, workspace_bytes=None,
+                      stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().gdn_state_step_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logit), _ptr(beta_logit),
+                                  _ptr(state), _ptr(out), B, H, T, d_k, d_v, frame_len, chunk_len,
+                                  _ptr(workspace), wb, _stream(stream))
+    return _check(st, "gdn_state_step_ws", check)
+
+
+def gdn_forward_host_ws(h_q, h_k, h_v, h_gate_logit, h_beta_logit, h_state_in, h_state_out, h_out,
+                        d_q, d_k, d_v, d_gate_logit, d_beta_logit, d_state, d_out,
+                        B, H, T, d_k_dim, d_v_dim, frame_len, chunk_len, workspace,
+                        workspace_bytes=None, stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().gdn_forward_host_ws(
+        _ptr(h_q), _ptr(h_k), _ptr(h_v), _ptr(h_gate_logit), _ptr(h_beta_logit),
+        _ptr(h_state_in), _ptr(h_state_out), _ptr(h_out),
+        _ptr(d_q), _ptr(d_k), _ptr(d_v), _ptr(d_gate_logit), _ptr(d_beta_logit),
+        _ptr(d_state), _ptr(d_out), B, H, T, d_k_dim, d_v_dim, frame_len, chunk_len,
+        _ptr(workspace), wb, _stream(stream))
+    return _check(st, "gdn_forward_host_ws", check)
+
+
 def gdn_get_last_device_status(stream=None) -> int:
     return load().gdn_get_last_device_status(_stream(stream))
 
@@ -159,30 +215,53 @@ def gdn_version() -> int:
 # tensor-level convenience wrappers (allocation by PyTorch, compute in the library)
 # ----------------------------------------------------------------------------
 
+def workspace(B, H, T, d_k, d_v, chunk_len=64, device="cuda"):
+    """A workspace tensor for the *_ws calls (None if these sizes need none)."""
+    import torch
+    n = gdn_workspace_bytes(B, H, T, d_k, d_v, chunk_len)
+    if n == 0:
+        return None
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
 def forward(q, k, v, gate_logit, beta_logit, state_in=None, frame_len=880, chunk_len=64,
-            want_state=True, stream=None):
+            want_state=True, stream=None, ws=None):
     """out, state_out = forward(q [B,T,H,dk], k, v [B,T,H,dv], gate [B,F,H], beta [B,T,H], ...).
 
-    bf16 q/k/v call gdn_forward, float32 q/k/v call gdn_forward_f32.
+    bf16 q/k/v call gdn_forward (gdn_forward_ws when a workspace ``ws`` is
+    given), float32 q/k/v call gdn_forward_f32.
     """
     import torch
     B, T, H, dk = q.shape
     dv = v.shape[3]
     out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     st = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_state else None
-    fn = gdn_forward_f32 if q.dtype == torch.float32 else gdn_forward
-    fn(q, k, v, gate_logit, beta_logit, state_in, st, out, B, H, T, dk, dv, frame_len,
-       chunk_len, stream)
+    if q.dtype == torch.float32:
+        gdn_forward_f32(q, k, v, gate_logit, beta_logit, state_in, st, out, B, H, T, dk, dv,
+                        frame_len, chunk_len, stream)
+    elif ws is not None:
+        gdn_forward_ws(q, k, v, gate_logit, beta_logit, state_in, st, out, B, H, T, dk, dv,
+                       frame_len, chunk_len, ws, stream=stream)
+    else:
+        gdn_forward(q, k, v, gate_logit, beta_logit, state_in, st, out, B, H, T, dk, dv,
+                    frame_len, chunk_len, stream)
     return out, st
 
 
 def state_step(q, k, v, gate_logit, beta_logit, state, frame_len=880, chunk_len=64,
-               want_out=True, stream=None):
+               want_out=True, stream=None, ws=None):
     """Advance ``state`` in place over one streaming block; returns out (or None)."""
     import torch
     B, T, H, dk = q.shape
     dv = v.shape[3]
     out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device) if want_out else None
-    fn = gdn_state_step_f32 if q.dtype == torch.float32 else gdn_state_step
-    fn(q, k, v, gate_logit, beta_logit, state, out, B, H, T, dk, dv, frame_len, chunk_len, stream)
+    if q.dtype == torch.float32:
+        gdn_state_step_f32(q, k, v, gate_logit, beta_logit, state, out, B, H, T, dk, dv,
+                           frame_len, chunk_len, stream)
+    elif ws is not None:
+        gdn_state_step_ws(q, k, v, gate_logit, beta_logit, state, out, B, H, T, dk, dv,
+                          frame_len, chunk_len, ws, stream=stream)
+    else:
+        gdn_state_step(q, k, v, gate_logit, beta_logit, state, out, B, H, T, dk, dv,
+                       frame_len, chunk_len, stream)
     return out

@@ -32,7 +32,8 @@
  * Ownership and memory.  The caller owns every buffer; device pointers must
  * point to device memory of the current device, host pointers (gdn_forward_host
  * only) should be pinned.  The library allocates no memory and keeps no state
- * between calls except one device status word per device.
+ * between calls except one device status word per device.  The *_ws entry
+ * points additionally take a caller-owned device workspace (see below).
  *
  * Asynchrony.  Work is enqueued on `stream` (0 = legacy default stream) and
  * the call returns without waiting, except gdn_forward_host, which waits for
@@ -117,12 +118,63 @@ int gdn_forward_host(const void* h_q, const void* h_k, const void* h_v,
                      int B, int H, int T, int d_k_dim, int d_v_dim,
                      int frame_len, int chunk_len, cudaStream_t stream);
 
+/*
+ * Workspace entry points.  The chunked method splits every chunk's work into a
+ * state-independent half (gates, norms, the decayed key Gram matrix, the UT
+ * inverse T = (I + A)^{-1} diag(beta), W = T diag(e^G) K and U = T V) and the
+ * state chain.  gdn_forward runs the first half once per 16 state columns;
+ * the *_ws calls run it once per chunk and head and hand the results to the
+ * CTAs of the head's state chain through a ring of records in `workspace`
+ * (a few tens of MB, sized by gdn_workspace_bytes, reused chunk after chunk so
+ * that it stays in L2).  Results equal gdn_forward's up to rounding.
+ *
+ * gdn_workspace_bytes writes to *bytes the workspace size the *_ws calls need
+ * for these sizes on the CURRENT device (it depends on the SM count); 0 means
+ * the sizes take a path without workspace (d_k or d_v <= 64, chunk_len != 64
+ * or T = 0) and `workspace` may then be NULL.  Returns a gdn_status.
+ *
+ * workspace: device memory of the current device, 256-byte aligned, at least
+ * *bytes long, overlapping no other argument.  Its contents need no
+ * initialisation and are garbage afterwards.  Calls that share a workspace
+ * must not run concurrently (same stream, or ordered by events).  Otherwise
+ * the arguments, layouts and errors are those of gdn_forward / gdn_state_step
+ * / gdn_forward_host; a too small, misaligned, NULL (when needed) or
+ * overlapping workspace gives GDN_ERR_INVALID_ARG.  The kernel is launched
+ * cooperatively (all of its CTAs resident at once); while another kernel
+ * occupies SMs of the device the launch may fail with GDN_ERR_CUDA.
+ */
+int gdn_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk_len, size_t* bytes);
+
+int gdn_forward_ws(const void* q, const void* k, const void* v,
+                   const float* gate_logit, const float* beta_logit,
+                   const float* state_in, float* state_out, void* out,
+                   int B, int H, int T, int d_k, int d_v,
+                   int frame_len, int chunk_len, void* workspace, size_t workspace_bytes,
+                   cudaStream_t stream);
+
+int gdn_state_step_ws(const void* q, const void* k, const void* v,
+                      const float* gate_logit, const float* beta_logit,
+                      float* state, void* out,
+                      int B, int H, int T, int d_k, int d_v,
+                      int frame_len, int chunk_len, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream);
+
+int gdn_forward_host_ws(const void* h_q, const void* h_k, const void* h_v,
+                        const float* h_gate_logit, const float* h_beta_logit,
+                        const float* h_state_in, float* h_state_out, void* h_out,
+                        void* d_q, void* d_k, void* d_v,
+                        float* d_gate_logit, float* d_beta_logit,
+                        float* d_state, void* d_out,
+                        int B, int H, int T, int d_k_dim, int d_v_dim,
+                        int frame_len, int chunk_len, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
 /* Human-readable text of a gdn_status value (static storage). */
 const char* gdn_status_string(int status);
 
 /*
  * Every wait inside the kernels (on an mbarrier completing a TMA copy or a
- * tensor-core MMA) is bounded.  A wait that runs out records GDN_ERR_TIMEOUT in
+ * tensor-core MMA, or on a ring flag written by another CTA) is bounded.  A wait that runs out records GDN_ERR_TIMEOUT in
  * a per-device status word and the kernel stops its work and returns cleanly.
  * This call synchronises `stream`, returns the recorded status (GDN_OK if none)
  * and clears it.

@@ -62,8 +62,9 @@ def assert_f32_parity(x, ref, what):
     return e_rel
 
 
-def run_library(inp, device, state_in=None, want_state=True, chunk_len=64, canary=True):
-    """Run gdn_forward (bf16) or gdn_forward_f32 through the C ABI.
+def run_library(inp, device, state_in=None, want_state=True, chunk_len=64, canary=True, ws=False):
+    """Run gdn_forward (bf16; gdn_forward_ws with a fresh workspace if `ws`) or
+    gdn_forward_f32 through the C ABI.
 
     Outputs are NaN-filled first and surrounded by guard bands filled with a
     sentinel; the guards must come back untouched and no NaN may remain.
@@ -86,8 +87,15 @@ def run_library(inp, device, state_in=None, want_state=True, chunk_len=64, canar
     st_buf[-guard:] = 7.0
     st = st_buf[guard:guard + n_st] if want_state else None
     s_in = None if state_in is None else f32_device(state_in, device)
-    fn = G.gdn_forward_f32 if inp.io_dtype == "f32" else G.gdn_forward
-    fn(q, k, v, g, b, s_in, st, out, Bn, H, T, dk, dv, inp.frame_len, chunk_len)
+    if ws and inp.io_dtype == "bf16":
+        wsp = G.workspace(Bn, H, T, dk, dv, chunk_len, device)
+        if wsp is not None:
+            wsp.fill_(0xA5)          # garbage: the call must not depend on its contents
+        G.gdn_forward_ws(q, k, v, g, b, s_in, st, out, Bn, H, T, dk, dv, inp.frame_len, chunk_len,
+                         wsp)
+    else:
+        fn = G.gdn_forward_f32 if inp.io_dtype == "f32" else G.gdn_forward
+        fn(q, k, v, g, b, s_in, st, out, Bn, H, T, dk, dv, inp.frame_len, chunk_len)
     torch.cuda.synchronize()
     assert G.gdn_get_last_device_status() == G.GDN_OK
     if canary:

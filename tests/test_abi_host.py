@@ -114,3 +114,37 @@ def test_binding_raises_on_error():
         G.gdn_forward(A, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 24, 32, 16, 16,
                       stream=0)
     assert e.value.status == G.GDN_ERR_UNSUPPORTED
+
+
+def test_workspace_size_query_validates():
+    import ctypes
+    lib = G.load()
+    n = ctypes.c_size_t(123)
+    assert lib.gdn_workspace_bytes(1, 2, 64, 32, 32, 64, None) == G.GDN_ERR_INVALID_ARG
+    assert lib.gdn_workspace_bytes(0, 2, 64, 112, 112, 64, ctypes.byref(n)) == G.GDN_ERR_INVALID_ARG
+    assert lib.gdn_workspace_bytes(1, 2, 64, 24, 112, 64, ctypes.byref(n)) == G.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_workspace_bytes(1, 2, 64, 112, 112, 48, ctypes.byref(n)) == G.GDN_ERR_UNSUPPORTED
+    # sizes served without a workspace answer 0 without touching the device
+    for dims in ((1, 2, 64, 32, 32, 64), (1, 2, 64, 112, 112, 32), (1, 2, 0, 112, 112, 64),
+                 (1, 2, 64, 64, 112, 64)):
+        n.value = 123
+        assert lib.gdn_workspace_bytes(*dims, ctypes.byref(n)) == G.GDN_OK
+        assert n.value == 0
+
+
+def test_workspace_entry_points_validate_first():
+    lib = G.load()
+    # argument errors come before any workspace or device check
+    st = lib.gdn_forward_ws(None, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 112,
+                            112, 16, 64, None, 0, None)
+    assert st == G.GDN_ERR_INVALID_ARG
+    st = lib.gdn_forward_ws(A, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 24,
+                            112, 16, 64, None, 0, None)
+    assert st == G.GDN_ERR_UNSUPPORTED
+    st = lib.gdn_state_step_ws(A, 2 * A, 3 * A, 4 * A, 5 * A, None, 6 * A, 1, 2, 64, 112, 112,
+                               16, 64, 7 * A, 1 << 20, None)
+    assert st == G.GDN_ERR_INVALID_ARG      # no state
+    # the host-buffer form refuses a missing workspace before copying anything
+    st = lib.gdn_forward_host_ws(A, A, A, A, A, None, None, A, A, 2 * A, 3 * A, 4 * A, 5 * A,
+                                 None, 6 * A, 1, 2, 64, 112, 112, 16, 64, None, 0, None)
+    assert st == G.GDN_ERR_INVALID_ARG
