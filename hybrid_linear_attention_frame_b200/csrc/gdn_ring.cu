@@ -19,7 +19,8 @@
 // publishes it with a GPU-scope release store.  Every CTA of the group runs the
 // chain for its own 16 columns over all chunks: a loader warp acquires the
 // record, pulls it into shared memory with bulk copies (plus the chunk's q and
-// k tiles by TMA) and reports the slot consumed once the copies have landed.
+// k tiles by TMA) and reports the slot consumed once the chain is done with it
+// (the loader publishes that, so that the chain warps never wait on a fence).
 // A producer re-fills a slot only after every CTA of the group has consumed
 // it.  Each wait depends only on chunks with a smaller index, and the launch is
 // cooperative (all CTAs resident), so the protocol cannot deadlock; every wait
@@ -28,8 +29,9 @@
 // Groups are persistent: group g serves chains g, g + G, g + 2G, ... back to
 // back, numbering their chunks consecutively.
 //
-// Warp roles inside a CTA: warps 0-3 run the chain, warps 4-11 the prep of
-// this CTA's share of the chunks, warp 12 loads the chain's records.
+// Warp roles inside a CTA: warps 0-3 run the state chain, warps 4-11 the prep
+// of this CTA's share of the chunks, warps 12-13 the intra-chunk product P E
+// and the output, warps 14 and 15 load the two parts of the chain's slots.
 #include <cudaTypedefs.h>
 
 #include "gdn_common.cuh"
@@ -44,11 +46,14 @@ using tc::kC;
 using tc::kXS;
 
 constexpr int kVB = 16;                // state columns per CTA
-constexpr int kThreads = 416;          // 13 warps
-constexpr int kChainThreads = 128;     // warps 0-3
-constexpr int kPrepThreads = 256;      // warps 4-11
-constexpr int kLoaderWarp = 12;
-constexpr uint32_t kBarChain = 1, kBarPrep = 2;   // named barriers (3 is the inverse's)
+constexpr int kThreads = 512;          // 16 warps
+constexpr int kChainThreads = 128;     // warps 0-3: the state chain
+constexpr int kPrepThreads = 256;      // warps 4-11: prep of this CTA's share of the chunks
+constexpr int kOutWarp0 = 12;          // warps 12, 13: P E and the output (TMEM lanes 0-63)
+constexpr int kLoaderA = 14;           // warp 14: part A of the chain's slots (q and W tiles)
+constexpr int kLoaderB = 15;           // warp 15: part B (k tile, P, U, scalars)
+// named barriers (3 is the UT inverse's)
+constexpr uint32_t kBarChain = 1, kBarPrep = 2, kBarPrepHi = 4, kBarOut = 6;
 constexpr int kRing = 16;              // record slots per group
 constexpr uint32_t kTmemCols = 512;
 
@@ -56,9 +61,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColG = 0;          // [K;Q][K;Q]^T     128 (prep)
 constexpr uint32_t kColW = 128;        // [T';T] K         128 (prep; lanes 0-63 = W)
 constexpr uint32_t kColU = 256;        // [T';T] V         128 (prep; lanes 64-127 = U)
-constexpr uint32_t kColQW = 384;       // [Q;W] S          16  (chain)
-constexpr uint32_t kColS = 400;        // K^T E'           16  (chain)
-constexpr uint32_t kColPE = 416;       // [P;X] E          2 x 16 (chain)
+constexpr uint32_t kColQW = 384;       // [Q;W] S          4 x 16 (chain, by chunk mod 4)
+constexpr uint32_t kColS = 448;        // K^T E'           16     (chain)
+constexpr uint32_t kColPE = 464;       // [P;X] E          2 x 16 (output warps, by chunk parity)
 
 // ---- record (global memory, one per ring slot) ----
 constexpr uint32_t kRecW = 0;          // W image: d-columns 0-63 | 64-127, 8 KB each (SW128)
@@ -92,17 +97,28 @@ constexpr uint32_t kOffTp = kOffPrep + 49152;
 constexpr uint32_t kOffT = kOffTp + kTile;
 constexpr uint32_t kOffAXI = kOffT + kTile;
 constexpr uint32_t kScFloats = 13 * 64 + 16;
-constexpr uint32_t kOffSc = kOffAXI + 64 * kXS * 4;
-constexpr uint32_t kOffSB = ((kOffSc + kScFloats * 4 + 255) / 256) * 256;   // S bf16, SW32
-constexpr uint32_t kOffEB = kOffSB + 128 * 32;     // E  bf16, SW32
-constexpr uint32_t kOffEP = kOffEB + 64 * 32;      // E' bf16, SW32
-constexpr uint32_t kOffBar = kOffEP + 64 * 32;
-// barriers: full[2], cfree[2] (chain ring), ptma, g1, wu (prep), m1, m2 (chain)
-constexpr uint32_t kBarFull = 0, kBarFree = 2, kBarPTma = 4, kBarG1 = 5, kBarWU = 6, kBarM1 = 7,
-                   kBarM2 = 8, kNumBars = 9;
+constexpr uint32_t kOffSc = kOffAXI + 64 * kXS * 4;   // prep scalars, 2 buffers (chunk parity)
+constexpr uint32_t kOffSB = ((kOffSc + 2 * kScFloats * 4 + 255) / 256) * 256;   // S bf16, SW32
+constexpr uint32_t kOffEB = kOffSB + 128 * 32;     // E  bf16, SW32, 2 buffers (chunk parity)
+constexpr uint32_t kOffEP = kOffEB + 2 * 64 * 32;  // E' bf16, SW32, 2 buffers
+constexpr uint32_t kOffBar = kOffEP + 2 * 64 * 32;
+// mbarriers.  A chain slot is filled in two parts: A = Q and W (read by MMA1 only, so
+// released as soon as MMA1 completes) and B = K, P, U and the scalars.
+//   fullA[2], fullB[2], freeA[2], freeB[2] (chain ring), ptma, g1, wu (prep), m1,
+//   m2s (K^T E'), m2p (P E), eready[2] (E of a slot's chunk is in shared memory and
+//   K^T E' has been issued)
+// (Loader A tells loader B how many records it has acquired through a monotonic
+// counter, not an mbarrier: A may run two chunks ahead of B, and an mbarrier
+// phase that advances twice between two looks of its waiter is ambiguous.)
+constexpr uint32_t kBarFullA = 0, kBarFullB = 2, kBarFreeA = 4, kBarFreeB = 6, kBarPTma = 8, kBarG1 = 9,
+                   kBarWU = 10, kBarM1 = 11, kBarM2S = 12, kBarM2P = 13, kBarEReady = 14, kNumBars = 16;
+constexpr uint32_t kFreeBArrivals = 3;  // chain thread 0, one lane of each output warp
+constexpr uint32_t kBytesA = 4 * 8192;                          // Q0, Q1, W0, W1
+constexpr uint32_t kBytesB = 2 * 8192 + 8192 + 4096 + 528;      // K0, K1, P, U slice, scalars
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
-constexpr uint32_t kSmemUsed = kOffAbort + 4;
+constexpr uint32_t kOffRecOk = kOffAbort + 4;      // records acquired by loader A (monotonic)
+constexpr uint32_t kSmemUsed = kOffRecOk + 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;
 
 // prep scalar table (floats)
@@ -185,8 +201,8 @@ __device__ __forceinline__ void gstore8_sw128(uint8_t* img, uint32_t row, uint32
 
 // Spin (bounded) until *flag >= want.  Gives up, raising both abort words and
 // recording `code`, after `limit_ns` or as soon as an abort word is raised.
-__device__ __forceinline__ bool wait_flag(const uint64_t* flag, uint64_t want, volatile int* abort_cta,
-                                          uint64_t* abort_glob, uint64_t limit_ns, int code) {
+__device__ __noinline__ bool wait_flag(const uint64_t* flag, uint64_t want, volatile int* abort_cta,
+                                       uint64_t* abort_glob, uint64_t limit_ns, int code) {
     if (ld_acquire_u64(flag) >= want) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
@@ -207,32 +223,143 @@ __device__ __forceinline__ bool wait_flag(const uint64_t* flag, uint64_t want, v
     }
 }
 
-// Where chunk n of group g lives: chain index and chunk within the chain.
+// Spin (bounded) until the shared-memory counter at `addr` reaches `want`.
+__device__ __noinline__ bool wait_counter(uint32_t addr, uint32_t want, volatile int* abort_cta, uint64_t limit_ns,
+                                          int code) {
+    if (ld_acquire_cta_shared(addr) >= want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(32);
+        if (ld_acquire_cta_shared(addr) >= want) return true;
+        if ((it & 15u) == 0) {
+            if (*abort_cta) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                *abort_cta = 1;
+                atomicCAS(&g_device_status, 0, code);
+                return false;
+            }
+        }
+    }
+}
+
+// The whole warp waits (bounded) until flags[v] >= want for every v < nflags, one
+// flag per lane, and returns in `known` the smallest value it saw (flags only
+// grow, so a later, smaller `want` needs no new reads).
+__device__ __forceinline__ bool wait_flags_warp(const uint64_t* flags, int nflags, uint64_t want, uint64_t& known,
+                                                volatile int* abort_cta, uint64_t* abort_glob, uint64_t limit_ns,
+                                                int code) {
+    const int lane = threadIdx.x & 31;
+    bool ok = true;
+    uint64_t seen = ~0ull;
+    if (lane < nflags) {
+        seen = ld_acquire_u64(flags + lane);
+        if (seen < want) {
+            ok = wait_flag(flags + lane, want, abort_cta, abort_glob, limit_ns, code);
+            seen = want;
+        }
+    }
+    ok = __all_sync(0xffffffffu, ok);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t o = __shfl_xor_sync(0xffffffffu, seen, off);
+        seen = o < seen ? o : seen;
+    }
+    known = seen;
+    return ok;
+}
+
+// Where a chunk of group g lives: chain x = (b, h), chunk c of that chain and
+// its valid length L.  Chunks of a group are numbered chain after chain, so a
+// cursor advances by a fixed stride without per-chunk divisions.
 struct Item {
-    int b, h, c, L;
+    int x, b, h, c, L;
 };
-__device__ __forceinline__ Item item_of(const FwdParams& p, int g, int G, int ntk, int n) {
-    Item it;
-    const int x = g + (n / ntk) * G;
+__device__ __forceinline__ void item_set(Item& it, const FwdParams& p, int x, int c) {
+    it.x = x;
     it.b = x / p.H;
-    it.h = x % p.H;
-    it.c = n % ntk;
-    it.L = min(kC, p.T - it.c * kC);
+    it.h = x - it.b * p.H;
+    it.c = c;
+    it.L = min(kC, p.T - c * kC);
+}
+// chunk n of group g (one division, for the start of a cursor)
+__device__ __forceinline__ Item item_at(const FwdParams& p, int g, int G, int ntk, int n) {
+    Item it;
+    const int k = n / ntk;
+    item_set(it, p, g + k * G, n - k * ntk);
     return it;
+}
+// advance by `step` chunks
+__device__ __forceinline__ void item_advance(Item& it, const FwdParams& p, int G, int ntk, int step) {
+    int c = it.c + step, x = it.x;
+    if (c >= ntk) {
+        while (c >= ntk) { c -= ntk; x += G; }
+        item_set(it, p, x, c);
+    } else {
+        it.c = c;
+        it.L = min(kC, p.T - c * kC);
+    }
 }
 
 
 // Bounded wait used only on the way out after an abort (async copies or MMAs
 // that may still be in flight must land before shared memory and TMEM go).
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+__device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < limit_ns) {
+    }
+}
+
+// Gates (G, beta) and decay tables of chunk jt into `scx`, run by the 128 prep
+// threads of warps pw 4-7 (out of line: it has two call sites).
+__device__ __noinline__ void prep_gates_tables(const FwdParams& p, const Item& jt, float* scx, int pw, int lane,
+                                               int pt) {
+    const int L = jt.L;
+    if (pw == 4) {
+        const int i0 = 2 * lane, i1 = i0 + 1, t0 = jt.c * kC + i0;
+        float g0 = 0.0f, g1 = 0.0f, r0 = 0.0f, r1 = 0.0f;
+        if (i0 < L) {
+            g0 = __ldg(p.gate + ((size_t)jt.b * p.F + t0 / p.frame_len) * p.H + jt.h);
+            r0 = __ldg(p.beta + ((size_t)jt.b * p.T + t0) * p.H + jt.h);
+        }
+        if (i1 < L) {
+            g1 = __ldg(p.gate + ((size_t)jt.b * p.F + (t0 + 1) / p.frame_len) * p.H + jt.h);
+            r1 = __ldg(p.beta + ((size_t)jt.b * p.T + t0 + 1) * p.H + jt.h);
+        }
+        const float la0 = (i0 < L) ? -softplus_fast(g0) : 0.0f;
+        const float la1 = (i1 < L) ? -softplus_fast(g1) : 0.0f;
+        float x = la0 + la1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        scx[SC_G + i0] = x - la1;
+        scx[SC_G + i1] = x;
+        scx[SC_BETA + i0] = (i0 < L) ? sigmoid_fast(r0) : 0.0f;
+        scx[SC_BETA + i1] = (i1 < L) ? sigmoid_fast(r1) : 0.0f;
+    }
+    named_bar_sync(kBarPrepHi, 128);
+    const float GL = scx[SC_G + L - 1];
+    for (int idx = pt - 128; idx < 256; idx += 128) {
+        if (idx < 64) {
+            const int i = idx;
+            const float Gi = scx[SC_G + i];
+            scx[SC_GAM + i] = __expf(Gi);
+            scx[SC_DL + i] = (i < L) ? __expf(GL - Gi) : 0.0f;     // times 1/|k_i| later
+            scx[SC_EXR + i] = (i >= 16) ? __expf(Gi - scx[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
+            if (i == 0) scx[SC_MISC] = __expf(GL);
+        } else {
+            const int bi = 1 + (idx - 64) / 64, j = idx & 63;
+            scx[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? __expf(scx[SC_G + 16 * bi - 1] - scx[SC_G + j]) : 0.0f;
+        }
     }
 }
 
 // ---------------------------------------------------------------- MMA issue (one warp)
 
 // prep: [K;Q][K;Q]^T (M = N = 128, K = d_k)
+// (K loops are unrolled to their maximum with a warp-uniform guard, so that the
+// descriptors are a base plus compile-time offsets)
 __device__ __forceinline__ void issue_g1(uint32_t prep, uint32_t tmem, int nks) {
     for (int ks = 0; ks < nks; ++ks) {
         const uint64_t a = kmaj128(dstep(prep + pK0, ks, kPHalf));
@@ -252,22 +379,30 @@ __device__ __forceinline__ void issue_wu(uint32_t prep, uint32_t tp, uint32_t tm
     }
 }
 
-// chain: [Q;W] S (M = 128, N = 16, K = d_k)
-__device__ __forceinline__ void issue_m1(uint32_t slot, uint32_t sb, uint32_t tmem, int nks) {
-    for (int ks = 0; ks < nks; ++ks)
-        mma_bf16_warp(tmem + kColQW, kmaj128(dstep(slot + cQ0, ks, kCHalfQ)), mnmaj32(sb + (uint32_t)ks * 512u),
-                      kIdM1, ks > 0);
+// chain: [Q;W] S (M = 128, N = 16, K = d_k) into accumulator buffer qb.  Four buffers:
+// MMA1 of chunk n + 4 can only start after the output warps released chunk n's slot.
+__device__ __forceinline__ void issue_m1(uint32_t slot, uint32_t sb, uint32_t tmem, int nks, int qb) {
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks)
+        if (ks < nks)
+            mma_bf16_warp(tmem + kColQW + 16u * qb, kmaj128(dstep(slot + cQ0, ks, kCHalfQ)),
+                          mnmaj32(sb + (uint32_t)ks * 512u), kIdM1, ks > 0);
 }
 
-// chain: K^T E' (M = 128 over d_k) and [P;X] E (rows 0-63 used), K = 64 tokens
-__device__ __forceinline__ void issue_m2(uint32_t slot, uint32_t eb, uint32_t ep, uint32_t tmem, int s) {
+// chain: K^T E' (M = 128 over d_k), K = 64 tokens: the state increment
+__device__ __forceinline__ void issue_m2s(uint32_t slot, uint32_t ep, uint32_t tmem) {
 #pragma unroll
-    for (int ks = 0; ks < kC / 16; ++ks) {
+    for (int ks = 0; ks < kC / 16; ++ks)
         mma_bf16_warp(tmem + kColS, mnmaj128(slot + cK0 + (uint32_t)ks * 2048u, kCHalfK),
                       mnmaj32(ep + (uint32_t)ks * 512u), kIdM2S, ks > 0);
+}
+
+// chain: [P;X] E (rows 0-63 used), K = 64 tokens: the intra-chunk part of the output
+__device__ __forceinline__ void issue_m2p(uint32_t slot, uint32_t eb, uint32_t tmem, int s) {
+#pragma unroll
+    for (int ks = 0; ks < kC / 16; ++ks)
         mma_bf16_warp(tmem + kColPE + 16u * s, kmaj128(slot + cP + (uint32_t)ks * 32u),
                       mnmaj32(eb + (uint32_t)ks * 512u), kIdM2P, ks > 0);
-    }
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -295,7 +430,7 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     float* AXI = reinterpret_cast<float*>(gb + kOffAXI);
     float* MSf = reinterpret_cast<float*>(gb + kOffT);
-    float* sc = reinterpret_cast<float*>(gb + kOffSc);
+    float* sc0 = reinterpret_cast<float*>(gb + kOffSc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + kOffAbort);
     const uint32_t bars = base + kOffBar;
     auto bar = [&](uint32_t i) { return bars + 8u * i; };
@@ -308,9 +443,11 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_relinquish();
     }
     if (tid == 32) {
-        for (uint32_t i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+        for (uint32_t i = 0; i < kNumBars; ++i)
+            mbar_init(bar(i), (i == kBarFreeB || i == kBarFreeB + 1) ? kFreeBArrivals : 1u);
         fence_mbar_init();
         *abort_flag = 0;
+        *reinterpret_cast<volatile uint32_t*>(gb + kOffRecOk) = 0u;
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
@@ -322,40 +459,22 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gb + kOffTmemSlot);
 
     if (warp < 4) {
-        // ======================= chain =======================
-        float S[16], QS[16];
-        float gq = 0.0f;
+        // ======================= chain (warps 0-3) =======================
+        // Per chunk n (slot and accumulator parity s = n & 1): MMA1 [Q;W] S ->
+        // E = U - W S (warps 2-3) -> K^T E' -> S update.  P E and the output are
+        // left to the output warps (eready[s] hands E over).
+        float S[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) { S[j] = 0.0f; QS[j] = 0.0f; }
-        bool ok = true, m1_pending = false, m2_pending = false;
-        int pend_n = -1;                      // item whose output is still to be written
-        Item pend{0, 0, 0, 0};
-        // O = diag(e^G/|q|) Q S + P E of item n (warps 0, 1; rows 32*qtr + lane)
-        auto output = [&](const Item& it, int n) {
-            if (qtr >= 2) return;
-            const int i = 32 * qtr + lane;
-            float pe[16];
-            tmem_ld16(tmem_lane(tmem, qtr) + kColPE + 16u * (uint32_t)(n & 1), pe);
-            tmem_wait_ld();
-            if (i < it.L && p.out) {
-                uint32_t w[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    w[j] = pack_bf16x2(fmaf(gq, QS[2 * j], pe[2 * j]), fmaf(gq, QS[2 * j + 1], pe[2 * j + 1]));
-                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) +
-                                   (((size_t)it.b * p.T + (size_t)it.c * kC + i) * p.H + it.h) * dv +
-                                   (size_t)vb * kVB;
-                uint4* o4 = reinterpret_cast<uint4*>(o);
-                o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            }
-        };
-        for (int n = 0; n < total; ++n) {
-            const Item it = item_of(p, g, G, ntk, n);
+        for (int j = 0; j < 16; ++j) S[j] = 0.0f;
+        bool ok = true;
+        int pending = -1;                      // barrier of an MMA group not yet waited for
+        Item it = item_at(p, g, G, ntk, 0);
+        for (int n = 0; n < total; ++n, item_advance(it, p, G, ntk, 1)) {
             const int s = n & 1;
             const uint32_t slot = base + (uint32_t)s * kCSlot;
             const float* csc = reinterpret_cast<const float*>(gb + (uint32_t)s * kCSlot + cSc);
             const float* cu = reinterpret_cast<const float*>(gb + (uint32_t)s * kCSlot + cU);
+            const uint32_t eb = ebt + (uint32_t)s * 2048u, ep = ept + (uint32_t)s * 2048u;
             if (it.c == 0) {
                 // first chunk of a chain: its initial state (this thread owns row tid)
                 const size_t sbase = ((size_t)it.b * p.H + it.h) * (size_t)dk * dv + (size_t)vb * kVB;
@@ -374,64 +493,55 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_before();
                 named_bar_sync(kBarChain, kChainThreads);
             }
-            ok = mbar_wait(bar(kBarFull + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 11);
+            ok = mbar_wait(bar(kBarFullA + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 11);
             if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
-            if (tid == 0) {
-                // the record is in shared memory: its ring slot may be re-filled
-                fence_proxy_async_global();
-                st_release_u64(consumed + vb, (uint64_t)n + 1);
-            }
             tc_fence_after();
             if (warp == 0) {
-                issue_m1(slot, sbt, tmem, nks);
+                issue_m1(slot, sbt, tmem, nks, n & 3);
                 mma_commit_warp(bar(kBarM1));
+                mma_commit_warp(bar(kBarFreeA + s));   // Q and W of the slot: read once MMA1 is done
             }
-            m1_pending = true;
-            if (it.c > 0) output(pend, pend_n);        // previous chunk's output while MMA1 runs
+            pending = kBarM1;
             ok = mbar_wait(bar(kBarM1), (uint32_t)(n & 1), abort_flag, lim, 4);
+            ok = ok && mbar_wait(bar(kBarFullB + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 15);
             if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
-            m1_pending = false;
+            pending = -1;
             tc_fence_after();
-            {
-                float v[16];
-                tmem_ld16(tmem_lane(tmem, qtr) + kColQW, v);
-                if (qtr < 2) {
-                    gq = csc[RS_GQ + 32 * qtr + lane];
-                    tmem_wait_ld();
+            if (qtr >= 2) {
+                const int i = 32 * (qtr - 2) + lane;
+                float v[16], u[16];
+                tmem_ld16(tmem_lane(tmem, qtr) + kColQW + 16u * (uint32_t)(n & 3), v);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) QS[j] = v[j];
-                } else {
-                    const int i = 32 * (qtr - 2) + lane;
-                    float u[16];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float4 u4 = ld4(cu + q * 256 + i * 4);
-                        u[4 * q] = u4.x; u[4 * q + 1] = u4.y; u[4 * q + 2] = u4.z; u[4 * q + 3] = u4.w;
-                    }
-                    const float d = csc[RS_DL + i];
-                    tmem_wait_ld();
-                    float e[16], e2[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        e[j] = u[j] - v[j];
-                        e2[j] = e[j] * d;
-                    }
-                    store_row16_sw32(ebt, (uint32_t)i, e);
-                    store_row16_sw32(ept, (uint32_t)i, e2);
+                for (int q = 0; q < 4; ++q) {
+                    const float4 u4 = ld4(cu + q * 256 + i * 4);
+                    u[4 * q] = u4.x; u[4 * q + 1] = u4.y; u[4 * q + 2] = u4.z; u[4 * q + 3] = u4.w;
                 }
+                const float d = csc[RS_DL + i];
+                tmem_wait_ld();
+                float e[16], e2[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    e[j] = u[j] - v[j];
+                    e2[j] = e[j] * d;
+                }
+                store_row16_sw32(eb, (uint32_t)i, e);
+                store_row16_sw32(ep, (uint32_t)i, e2);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(kBarChain, kChainThreads);
             if (warp == 0) {
                 tc_fence_after();
-                issue_m2(slot, ebt, ept, tmem, s);
-                mma_commit_warp(bar(kBarM2));
+                issue_m2s(slot, ep, tmem);
+                mma_commit_warp(bar(kBarM2S));
+                tc_fence_before();
+                if (elect_one()) mbar_arrive(bar(kBarEReady + s));
+                __syncwarp();
             }
-            m2_pending = true;
-            ok = mbar_wait(bar(kBarM2), (uint32_t)(n & 1), abort_flag, lim, 5);
+            pending = kBarM2S;
+            ok = mbar_wait(bar(kBarM2S), (uint32_t)(n & 1), abort_flag, lim, 5);
             if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
-            m2_pending = false;
+            pending = -1;
             tc_fence_after();
             {
                 float v[16];
@@ -445,36 +555,34 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(kBarChain, kChainThreads);
-            if (tid == 0) mbar_arrive(bar(kBarFree + s));   // slot s back to the loader
-            pend = it;
-            pend_n = n;
-            if (it.c == ntk - 1) {
-                // last chunk of the chain: its output and the final state
-                output(it, n);
-                if (p.state_out && tid < dk) {
-                    const size_t sbase = ((size_t)it.b * p.H + it.h) * (size_t)dk * dv + (size_t)vb * kVB;
-                    float4* so = reinterpret_cast<float4*>(p.state_out + sbase + (size_t)tid * dv);
+            if (tid == 0) mbar_arrive(bar(kBarFreeB + s));   // U, scalars and K of the slot are done with
+            if (it.c == ntk - 1 && p.state_out && tid < dk) {
+                // last chunk of the chain: the final state
+                const size_t sbase = ((size_t)it.b * p.H + it.h) * (size_t)dk * dv + (size_t)vb * kVB;
+                float4* so = reinterpret_cast<float4*>(p.state_out + sbase + (size_t)tid * dv);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        so[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
-                }
+                for (int j = 0; j < 4; ++j) so[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
             }
         }
-        if (!ok && (m1_pending || m2_pending)) {
-            // one parity is already complete, the other waits for the MMAs still in flight
-            const uint32_t mb = bar(m1_pending ? kBarM1 : kBarM2);
-            drain_wait(mb, 0, lim);
-            drain_wait(mb, 1, lim);
+        if (!ok && pending >= 0) {
+            // MMAs possibly still in flight must finish before TMEM is released
+            drain_wait(bar((uint32_t)pending), 0, lim);
+            drain_wait(bar((uint32_t)pending), 1, lim);
         }
     } else if (warp < 12) {
-        // ======================= prep =======================
+        // ======================= prep (warps 4-11) =======================
+        // Chunks vb, vb + ncb, vb + 2 ncb, ... of the group.  Overlapped with the
+        // current chunk: the next chunk's tiles (fetched once WU has consumed the
+        // current ones), its Gram matrices (started when the current record is
+        // handed to the publisher) and its gates and decay tables (computed by
+        // warps 8-11 while warps 4-7 run the UT inverse).
         const int pt = tid - kChainThreads;   // 0..255
         const int pw = warp - 4;              // 0..7
         bool ok = true;
         int mma_pending = -1;                 // barrier of an MMA group not yet waited for
         int ptma_issued = 0, ptma_waited = 0;
-        auto issue_prep_tma = [&](int nn) {
-            const Item jt = item_of(p, g, G, ntk, nn);
+        uint64_t cons_known = 0;              // all CTAs of the group have consumed this many chunks
+        auto issue_prep_tma = [&](const Item& jt) {
             const uint32_t pb = bar(kBarPTma);
             const int t0 = jt.c * kC;
             mbar_arrive_expect_tx(pb, 6 * kTile);
@@ -485,72 +593,43 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_load_4d(prep + pV0, &tm_v, pb, 0, jt.h, t0, jt.b);
             tma_load_4d(prep + pV1, &tm_v, pb, 64, jt.h, t0, jt.b);
         };
+        // Gram matrices of the chunk whose tiles are in flight (warp pw 4)
+        auto start_g1 = [&](int mm) -> bool {
+            if (!mbar_wait(bar(kBarPTma), (uint32_t)(mm & 1), abort_flag, lim, 1)) return false;
+            tc_fence_after();
+            issue_g1(prep, tmem, nks);
+            mma_commit_warp(bar(kBarG1));
+            return true;
+        };
+        auto gates_tables = [&](const Item& jt, float* scx) { prep_gates_tables(p, jt, scx, pw, lane, pt); };
+        Item it{0, 0, 0, 0, 0};
         if (vb < total) {
-            if (pw == 4 && elect_one()) issue_prep_tma(vb);
-            ptma_issued = 1;
+            it = item_at(p, g, G, ntk, vb);
+            if (pw == 4) {
+                if (elect_one()) issue_prep_tma(it);
+                __syncwarp();
+                ptma_issued = 1;
+                ok = start_g1(0);
+                if (ok) ptma_waited = 1;
+            }
+            if (pw >= 4) gates_tables(it, sc0);
+            mma_pending = ok ? (int)kBarG1 : -1;
         }
         int m = 0;
         for (int n = vb; n < total; n += ncb, ++m) {
-            const Item it = item_of(p, g, G, ntk, n);
-            const int L = it.L;
+            float* sc = sc0 + (m & 1) * kScFloats;
+            float* scn = sc0 + ((m + 1) & 1) * kScFloats;
             uint8_t* rec = recs + (size_t)(n % kRing) * recb;
+            Item nx = it;
+            item_advance(nx, p, G, ntk, ncb);
+            const bool has_next = n + ncb < total;
             // ---- the ring slot must have been consumed by every CTA of the group ----
-            bool got = true;
-            if (pt == 0 && n >= kRing)
-                for (int v = 0; v < ncb && got; ++v)
-                    got = wait_flag(consumed + v, (uint64_t)(n - kRing + 1), abort_flag, abort_glob, lim, 14);
-            // ---- gates: G (cumulative log-gate), beta ----
-            if (pw == 0) {
-                const int i0 = 2 * lane, i1 = i0 + 1, t0 = it.c * kC + i0;
-                float g0 = 0.0f, g1 = 0.0f, r0 = 0.0f, r1 = 0.0f;
-                if (i0 < L) {
-                    g0 = __ldg(p.gate + ((size_t)it.b * p.F + t0 / p.frame_len) * p.H + it.h);
-                    r0 = __ldg(p.beta + ((size_t)it.b * p.T + t0) * p.H + it.h);
-                }
-                if (i1 < L) {
-                    g1 = __ldg(p.gate + ((size_t)it.b * p.F + (t0 + 1) / p.frame_len) * p.H + it.h);
-                    r1 = __ldg(p.beta + ((size_t)it.b * p.T + t0 + 1) * p.H + it.h);
-                }
-                const float la0 = (i0 < L) ? -softplus_fast(g0) : 0.0f;
-                const float la1 = (i1 < L) ? -softplus_fast(g1) : 0.0f;
-                float x = la0 + la1;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, off);
-                    if (lane >= off) x += y;
-                }
-                sc[SC_G + i0] = x - la1;
-                sc[SC_G + i1] = x;
-                sc[SC_BETA + i0] = (i0 < L) ? sigmoid_fast(r0) : 0.0f;
-                sc[SC_BETA + i1] = (i1 < L) ? sigmoid_fast(r1) : 0.0f;
-            }
-            if (!group_all(kBarPrep, kPrepThreads, got)) { ok = false; break; }
-            {
-                const float GL = sc[SC_G + L - 1];
-                if (pt < 64) {
-                    const int i = pt;
-                    const float Gi = sc[SC_G + i];
-                    sc[SC_GAM + i] = __expf(Gi);
-                    sc[SC_DL + i] = (i < L) ? __expf(GL - Gi) : 0.0f;     // times 1/|k_i| below
-                    sc[SC_EXR + i] = (i >= 16) ? __expf(Gi - sc[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
-                    if (i == 0) sc[SC_MISC] = __expf(GL);
-                } else {
-                    const int idx = pt - 64;                  // 0..191
-                    const int bi = 1 + idx / 64, j = idx & 63;
-                    sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? __expf(sc[SC_G + 16 * bi - 1] - sc[SC_G + j]) : 0.0f;
-                }
-            }
-            // ---- [K;Q][K;Q]^T ----
-            ok = mbar_wait(bar(kBarPTma), (uint32_t)(m & 1), abort_flag, lim, 1);
-            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
-            ptma_waited = m + 1;
-            if (pw == 4) {
-                tc_fence_after();
-                issue_g1(prep, tmem, nks);
-                mma_commit_warp(bar(kBarG1));
-            }
-            mma_pending = kBarG1;
-            ok = mbar_wait(bar(kBarG1), (uint32_t)(m & 1), abort_flag, lim, 2);
+            bool got = ok;
+            if (pw == 0 && n >= kRing && cons_known < (uint64_t)(n - kRing + 1))
+                got = wait_flags_warp(consumed, ncb, (uint64_t)(n - kRing + 1), cons_known, abort_flag, abort_glob,
+                                      lim, 14) && ok;
+            // ---- [K;Q][K;Q]^T (started earlier); gates and tables are in sc ----
+            ok = got && mbar_wait(bar(kBarG1), (uint32_t)(m & 1), abort_flag, lim, 2);
             if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
             mma_pending = -1;
             tc_fence_after();
@@ -590,28 +669,27 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int bi = i >> 4;
                 const float Gi = sc[SC_G + i], exr = sc[SC_EXR + i];
                 const float ri = (qtr < 2) ? sc[SC_BETA + i] * sc[SC_RK + i] : sc[SC_RQ + i];
-#pragma unroll
+#pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     const int j0 = 32 * ch + 16 * hh;
-                    float v[16], gj[16], rkj[16], ex[16];
+                    float v[16], val[16];
                     tmem_ld16(tmem_lane(tg, qtr) + (uint32_t)j0, v);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         const float4 a = ld4(sc + SC_G + j0 + 4 * q4);
                         const float4 r4 = ld4(sc + SC_RK + j0 + 4 * q4);
                         const float4 e4 = ld4(sc + SC_EXC + 64 * bi + j0 + 4 * q4);
-                        gj[4 * q4] = a.x; gj[4 * q4 + 1] = a.y; gj[4 * q4 + 2] = a.z; gj[4 * q4 + 3] = a.w;
-                        rkj[4 * q4] = r4.x; rkj[4 * q4 + 1] = r4.y; rkj[4 * q4 + 2] = r4.z; rkj[4 * q4 + 3] = r4.w;
-                        ex[4 * q4] = e4.x; ex[4 * q4 + 1] = e4.y; ex[4 * q4 + 2] = e4.z; ex[4 * q4 + 3] = e4.w;
-                    }
-                    tmem_wait_ld();
-                    float val[16];
+                        const float gj[4] = {a.x, a.y, a.z, a.w};
+                        const float rkj[4] = {r4.x, r4.y, r4.z, r4.w};
+                        const float ex[4] = {e4.x, e4.y, e4.z, e4.w};
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int j = j0 + jj;
-                        const float dec = ((j >> 4) == bi) ? __expf(Gi - gj[jj]) : exr * ex[jj];
-                        const bool keep = (qtr < 2) ? (j < i) : (j <= i);
-                        val[jj] = keep ? ri * rkj[jj] * v[jj] * dec : 0.0f;
+                        for (int e = 0; e < 4; ++e) {
+                            const int jj = 4 * q4 + e, j = j0 + jj;
+                            const float dec = ((j >> 4) == bi) ? __expf(Gi - gj[e]) : exr * ex[e];
+                            const bool keep = (qtr < 2) ? (j < i) : (j <= i);
+                            val[jj] = keep ? ri * rkj[e] * v[jj] * dec : 0.0f;
+                        }
                     }
                     if (qtr < 2) {
 #pragma unroll
@@ -629,7 +707,7 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // ---- T = (I + A)^{-1} diag(beta), T' = T diag(e^G / |k|) ----
                 tc::unit_lower_inverse_64(AXI, MSf, pt);
                 const int i = pt >> 1, j0 = 32 * (pt & 1);
-#pragma unroll
+#pragma unroll 1
                 for (int q = 0; q < 2; ++q) {
                     const int jb = j0 + 16 * q;
                     float tv[16], tpv[16];
@@ -654,7 +732,7 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     store8_sw128(base + kOffTp, (uint32_t)i, (uint32_t)jb + 8, &tpv[8]);
                 }
             } else {
-                // ---- the chain's per-token scalars into the record ----
+                // ---- the chain's per-token scalars into the record; next chunk's gates ----
                 float* rs = reinterpret_cast<float*>(rec + rec_sc(dv));
                 const int j = pt - 128;
                 if (j < 64) {
@@ -663,6 +741,7 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 } else if (j < 68) {
                     rs[RS_GL + (j - 64)] = (j == 64) ? sc[SC_MISC] : 0.0f;
                 }
+                if (has_next) gates_tables(nx, scn);
             }
             fence_proxy_async_smem();
             named_bar_sync(kBarPrep, kPrepThreads);
@@ -676,92 +755,165 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
             mma_pending = -1;
             tc_fence_after();
-            // the prep tiles are free: fetch the next item's
-            if (pw == 4 && n + ncb < total) {
+            // the prep tiles are free: fetch the next chunk's
+            if (pw == 4 && has_next) {
                 if (elect_one()) {
                     fence_proxy_async_smem();
-                    issue_prep_tma(n + ncb);
+                    issue_prep_tma(nx);
                 }
                 __syncwarp();
+                ptma_issued = m + 2;
             }
-            if (n + ncb < total) ptma_issued = m + 2;
             // ---- W (TMEM lanes 0-63) and U (lanes 64-127) into the record ----
             {
                 const int half = pw >> 2;
-                if (qtr < 2) {
-                    const int i = 32 * qtr + lane;
-                    for (int cb = 64 * half; cb < 64 * half + 64 && cb < dk; cb += 16) {
-                        float v[16];
-                        tmem_ld16(tmem_lane(tmem, qtr) + kColW + (uint32_t)cb, v);
-                        tmem_wait_ld();
-                        uint8_t* img = rec + kRecW + (cb >= 64 ? kTile : 0u);
-                        gstore8_sw128(img, (uint32_t)i, (uint32_t)(cb & 63), &v[0]);
-                        gstore8_sw128(img, (uint32_t)i, (uint32_t)(cb & 63) + 8, &v[8]);
-                    }
-                } else {
-                    const int i = 32 * (qtr - 2) + lane;
-                    for (int cb = 64 * half; cb < 64 * half + 64 && cb < dv; cb += 16) {
-                        float v[16];
-                        tmem_ld16(tmem_lane(tmem, qtr) + kColU + (uint32_t)cb, v);
-                        tmem_wait_ld();
-                        uint8_t* dst = rec + kRecU + (uint32_t)(cb / 16) * 4096u + (uint32_t)i * 16u;
+                const bool wpart = qtr < 2;
+                const int i = wpart ? 32 * qtr + lane : 32 * (qtr - 2) + lane;
+                const int ncol = wpart ? dk : dv;
+                const uint32_t col0 = (wpart ? kColW : kColU) + 64u * (uint32_t)half;
+#pragma unroll 1
+                for (int q2 = 0; q2 < 4; q2 += 2) {
+                    float v[2][16];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            st_global_v4(dst + q * 1024, __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                                         __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+                    for (int q = 0; q < 2; ++q)
+                        if (64 * half + 16 * (q2 + q) < ncol)
+                            tmem_ld16(tmem_lane(tmem, qtr) + col0 + 16u * (q2 + q), v[q]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int cb = 64 * half + 16 * (q2 + q);
+                        if (cb >= ncol) continue;
+                        if (wpart) {
+                            uint8_t* img = rec + kRecW + (half ? kTile : 0u);
+                            gstore8_sw128(img, (uint32_t)i, (uint32_t)(16 * (q2 + q)), &v[q][0]);
+                            gstore8_sw128(img, (uint32_t)i, (uint32_t)(16 * (q2 + q) + 8), &v[q][8]);
+                        } else {
+                            uint8_t* dst = rec + kRecU + (uint32_t)(cb / 16) * 4096u + (uint32_t)i * 16u;
+#pragma unroll
+                            for (int r = 0; r < 4; ++r)
+                                st_global_v4(dst + r * 1024, __float_as_uint(v[q][4 * r]),
+                                             __float_as_uint(v[q][4 * r + 1]), __float_as_uint(v[q][4 * r + 2]),
+                                             __float_as_uint(v[q][4 * r + 3]));
+                        }
                     }
                 }
             }
             tc_fence_before();
-            named_bar_sync(kBarPrep, kPrepThreads);
+            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
             if (pt == 0) {
-                // publish: every write of the record happens-before the release, and
-                // is ordered before the consumers' bulk copies (async proxy)
-                __threadfence();
+                // publish: the barrier orders every prep thread's record writes before this
+                // thread's release; the proxy fence orders them before the consumers' bulk
+                // copies (async proxy)
                 fence_proxy_async_global();
                 st_release_u64(ready + (n % kRing), (uint64_t)n + 1);
             }
+            if (has_next) {
+                // next chunk's Gram matrices while its record slot is awaited
+                if (pw == 4) {
+                    ok = start_g1(m + 1);
+                    if (ok) ptma_waited = m + 2;
+                }
+                mma_pending = ok ? (int)kBarG1 : -1;
+            }
+            it = nx;
         }
         if (!ok) {
             if (pw == 4) {
                 if (ptma_issued > ptma_waited) drain_wait(bar(kBarPTma), (uint32_t)((ptma_issued - 1) & 1), lim);
-                if (mma_pending >= 0) {
-                    drain_wait(bar((uint32_t)mma_pending), 0, lim);
-                    drain_wait(bar((uint32_t)mma_pending), 1, lim);
-                }
+                if (mma_pending >= 0) drain_wait(bar((uint32_t)mma_pending), (uint32_t)(m & 1), lim);
             }
         }
-    } else {
-        // ======================= record loader (warp 12) =======================
-        bool ok = true;
-        int issued = 0;
-        for (int n = 0; n < total; ++n) {
+    } else if (warp < kLoaderA) {
+        // ======================= output (warps 12, 13: TMEM lanes 0-63) =======================
+        // For chunk n: P E (issued once the chain has written E and issued K^T E'),
+        // then O = diag(e^G/|q|) Q S + P E for rows 32*qtr + lane.
+        bool ok = true, m2p_pending = false;
+        Item it = item_at(p, g, G, ntk, 0);
+        const int i = 32 * qtr + lane;
+        for (int n = 0; n < total; ++n, item_advance(it, p, G, ntk, 1)) {
             const int s = n & 1;
+            const uint32_t slot = base + (uint32_t)s * kCSlot;
+            const float* csc = reinterpret_cast<const float*>(gb + (uint32_t)s * kCSlot + cSc);
+            ok = mbar_wait(bar(kBarEReady + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 7);
+            if (!group_all(kBarOut, 64, ok)) { ok = false; break; }
+            tc_fence_after();
+            const float gq = csc[RS_GQ + i];
+            if (warp == kOutWarp0) {
+                issue_m2p(slot, ebt + (uint32_t)s * 2048u, tmem, s);
+                mma_commit_warp(bar(kBarM2P));
+            }
+            m2p_pending = true;
+            ok = mbar_wait(bar(kBarM2P), (uint32_t)(n & 1), abort_flag, lim, 6);
+            if (!group_all(kBarOut, 64, ok)) { ok = false; break; }
+            m2p_pending = false;
+            tc_fence_after();
+            float qs[16], pe[16];
+            tmem_ld16(tmem_lane(tmem, qtr) + kColQW + 16u * (uint32_t)(n & 3), qs);
+            tmem_ld16(tmem_lane(tmem, qtr) + kColPE + 16u * (uint32_t)s, pe);
+            tmem_wait_ld();
+            if (i < it.L && p.out) {
+                uint32_t w[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    w[j] = pack_bf16x2(fmaf(gq, qs[2 * j], pe[2 * j]), fmaf(gq, qs[2 * j + 1], pe[2 * j + 1]));
+                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) +
+                                   (((size_t)it.b * p.T + (size_t)it.c * kC + i) * p.H + it.h) * dv +
+                                   (size_t)vb * kVB;
+                uint4* o4 = reinterpret_cast<uint4*>(o);
+                o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarFreeB + s));   // P, E and this chunk's TMEM are done with
+        }
+        if (!ok && m2p_pending && warp == kOutWarp0) {
+            drain_wait(bar(kBarM2P), 0, lim);
+            drain_wait(bar(kBarM2P), 1, lim);
+        }
+    } else if (warp == kLoaderA) {
+        // ======================= loader A (warp 14): q and W tiles =======================
+        // Part A of chunk n goes into slot s once MMA1 of chunk n - 2 has read the
+        // slot's part A, so it runs about two chunks ahead of the chain.  Ready flags
+        // are polled 16 chunks at a time (one L2 round trip and one proxy fence per
+        // batch while the prep is ahead), then loader B is told the record is ready.
+        bool ok = true;
+        int issued = 0, ready_upto = 0;
+        Item it = item_at(p, g, G, ntk, 0);
+        for (int n = 0; n < total; ++n, item_advance(it, p, G, ntk, 1)) {
+            const int s = n & 1;
+            if (n >= ready_upto) {
+                const int j = n + lane;
+                bool rdy = true;
+                if (lane == 0) {
+                    rdy = wait_flag(ready + (n % kRing), (uint64_t)n + 1, abort_flag, abort_glob, lim, 13);
+                } else if (lane < kRing && j < total) {
+                    rdy = ld_acquire_u64(ready + (j % kRing)) >= (uint64_t)j + 1;
+                } else {
+                    rdy = false;
+                }
+                if (!__shfl_sync(0xffffffffu, rdy ? 1 : 0, 0)) { ok = false; break; }
+                // chunks n .. n + run - 1 are ready (run >= 1: lanes in order up to the first not ready)
+                const uint32_t notready = __ballot_sync(0xffffffffu, !rdy);
+                ready_upto = n + (notready ? __ffs(notready) - 1 : 32);
+                __syncwarp();                 // orders every lane's acquire before lane 0's copies
+                fence_proxy_async_global();
+            }
             if (n >= 2) {
-                ok = mbar_wait(bar(kBarFree + s), (uint32_t)(((n >> 1) - 1) & 1), abort_flag, lim, 12);
+                ok = mbar_wait(bar(kBarFreeA + s), (uint32_t)(((n >> 1) - 1) & 1), abort_flag, lim, 12);
                 if (!ok) break;
             }
-            bool got = true;
-            if (lane == 0) got = wait_flag(ready + (n % kRing), (uint64_t)n + 1, abort_flag, abort_glob, lim, 13);
-            got = __shfl_sync(0xffffffffu, got, 0);
-            if (!got) { ok = false; break; }
             if (lane == 0) {
-                fence_proxy_async_global();
-                const Item it = item_of(p, g, G, ntk, n);
                 const uint8_t* rec = recs + (size_t)(n % kRing) * recb;
                 const uint32_t slot = base + (uint32_t)s * kCSlot;
-                const uint32_t fb = bar(kBarFull + s);
+                const uint32_t fa = bar(kBarFullA + s);
                 const int t0 = it.c * kC;
-                mbar_arrive_expect_tx(fb, 3 * kTile + 4096u + kScCopy + 4 * kTile);
-                bulk_load(slot + cW0, rec + kRecW, kTile, fb);
-                bulk_load(slot + cW1, rec + kRecW + kTile, kTile, fb);
-                bulk_load(slot + cP, rec + kRecP, kTile, fb);
-                bulk_load(slot + cU, rec + kRecU + (uint32_t)vb * 4096u, 4096u, fb);
-                bulk_load(slot + cSc, rec + rec_sc(dv), kScCopy, fb);
-                tma_load_4d(slot + cQ0, &tm_q, fb, 0, it.h, t0, it.b);
-                tma_load_4d(slot + cQ1, &tm_q, fb, 64, it.h, t0, it.b);
-                tma_load_4d(slot + cK0, &tm_k, fb, 0, it.h, t0, it.b);
-                tma_load_4d(slot + cK1, &tm_k, fb, 64, it.h, t0, it.b);
+                mbar_arrive_expect_tx(fa, kBytesA);
+                bulk_load(slot + cW0, rec + kRecW, kTile, fa);
+                bulk_load(slot + cW1, rec + kRecW + kTile, kTile, fa);
+                tma_load_4d(slot + cQ0, &tm_q, fa, 0, it.h, t0, it.b);
+                tma_load_4d(slot + cQ1, &tm_q, fa, 64, it.h, t0, it.b);
+                st_release_cta_shared(base + kOffRecOk, (uint32_t)(n + 1));
             }
             __syncwarp();
             issued = n + 1;
@@ -769,7 +921,44 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!ok && lane == 0) {
             // copies still in flight must land before shared memory goes away
             for (int n = max(0, issued - 2); n < issued; ++n)
-                drain_wait(bar(kBarFull + (n & 1)), (uint32_t)((n >> 1) & 1), lim);
+                drain_wait(bar(kBarFullA + (n & 1)), (uint32_t)((n >> 1) & 1), lim);
+        }
+        __syncwarp();
+    } else {
+        // ======================= loader B (warp 15): k tile, P, U, scalars =======================
+        // Part B of chunk n goes into slot s once chunk n - 2 is done with entirely (chain
+        // and output warps).  Then chunks 0 .. n - 2 count as consumed for the producers.
+        bool ok = true;
+        int issued = 0;
+        Item it = item_at(p, g, G, ntk, 0);
+        for (int n = 0; n < total; ++n, item_advance(it, p, G, ntk, 1)) {
+            const int s = n & 1;
+            ok = wait_counter(base + kOffRecOk, (uint32_t)(n + 1), abort_flag, lim, 16);
+            if (ok && n >= 2) ok = mbar_wait(bar(kBarFreeB + s), (uint32_t)(((n >> 1) - 1) & 1), abort_flag, lim, 12);
+            if (!ok) break;
+            if (lane == 0) {
+                fence_proxy_async_global();
+                const uint8_t* rec = recs + (size_t)(n % kRing) * recb;
+                const uint32_t slot = base + (uint32_t)s * kCSlot;
+                const uint32_t fbb = bar(kBarFullB + s);
+                const int t0 = it.c * kC;
+                mbar_arrive_expect_tx(fbb, kBytesB);
+                tma_load_4d(slot + cK0, &tm_k, fbb, 0, it.h, t0, it.b);
+                tma_load_4d(slot + cK1, &tm_k, fbb, 64, it.h, t0, it.b);
+                bulk_load(slot + cP, rec + kRecP, kTile, fbb);
+                bulk_load(slot + cU, rec + kRecU + (uint32_t)vb * 4096u, 4096u, fbb);
+                bulk_load(slot + cSc, rec + rec_sc(dv), kScCopy, fbb);
+                if (n >= 2 && ((n & 1) == 0 || n + 1 == total)) {
+                    // chunk n - 2 is done with, and its bulk copies had landed long before
+                    st_release_u64(consumed + vb, (uint64_t)(n - 1));
+                }
+            }
+            __syncwarp();
+            issued = n + 1;
+        }
+        if (!ok && lane == 0) {
+            for (int n = max(0, issued - 2); n < issued; ++n)
+                drain_wait(bar(kBarFullB + (n & 1)), (uint32_t)((n >> 1) & 1), lim);
         }
         __syncwarp();
     }
