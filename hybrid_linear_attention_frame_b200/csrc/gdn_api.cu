@@ -152,7 +152,7 @@ int forward_host(const void* h_q, const void* h_k, const void* h_v,
     if (e == cudaSuccess) e = cudaMemcpyAsync(d_beta_logit, h_beta_logit, nb, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess && h_state_in) e = cudaMemcpyAsync(d_state, h_state_in, ns, cudaMemcpyHostToDevice, stream);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
-    st = run_bf16_ws(p, chunk_len, ws, ws_bytes, stream);
+    st = ws ? run_bf16_ws(p, chunk_len, ws, ws_bytes, stream) : run_bf16(p, chunk_len, stream);
     if (st != GDN_OK) return st;
     e = cudaMemcpyAsync(h_out, d_out, nv, cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess && h_state_out) e = cudaMemcpyAsync(h_state_out, d_state, ns, cudaMemcpyDeviceToHost, stream);
