@@ -17,6 +17,7 @@ bool ring_supported(int dk, int dv, int chunk_len);
 cudaError_t ring_groups(int BH, int dv, int* groups);
 size_t ring_workspace_bytes(int G, int dv);
 cudaError_t launch_ring(const FwdParams& p, void* ws, size_t ws_bytes, cudaStream_t stream);
+cudaError_t static_scratch(void** ptr, size_t* bytes);
 int read_and_clear_device_status(cudaStream_t stream);
 }  // namespace gdn
 
@@ -246,6 +247,27 @@ int gdn_forward_host_ws(const void* h_q, const void* h_k, const void* h_v,
     return forward_host(h_q, h_k, h_v, h_gate_logit, h_beta_logit, h_state_in, h_state_out, h_out, d_q, d_k,
                         d_v, d_gate_logit, d_beta_logit, d_state, d_out, B, H, T, d_k_dim, d_v_dim, frame_len,
                         chunk_len, workspace, workspace_bytes, stream);
+}
+
+int gdn_forward_static_ws(const void* q, const void* k, const void* v,
+                          const float* gate_logit, const float* beta_logit,
+                          const float* state_in, float* state_out, void* out,
+                          int B, int H, int T, int d_k, int d_v,
+                          int frame_len, int chunk_len, cudaStream_t stream)
+{
+    gdn::FwdParams p;
+    int st = validate(q, k, v, gate_logit, beta_logit, state_in, state_out, out, true, 2,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
+    if (st != GDN_OK) return st;
+    if (!uses_ring(T, d_k, d_v, chunk_len)) return run_bf16(p, chunk_len, stream);
+    size_t need = 0;
+    st = workspace_need(B, H, d_v, &need);
+    if (st != GDN_OK) return st;
+    void* ws = nullptr;
+    size_t ws_bytes = 0;
+    if (gdn::static_scratch(&ws, &ws_bytes) != cudaSuccess) return GDN_ERR_CUDA;
+    if (need > ws_bytes) return GDN_ERR_UNSUPPORTED;     // more than the static scratch holds
+    return to_status(gdn::launch_ring(p, ws, ws_bytes, stream));
 }
 
 int gdn_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk_len, size_t* bytes)

@@ -1011,6 +1011,32 @@ size_t ring_workspace_bytes(int G, int dv)
     return ring::flags_bytes(G) + (size_t)G * ring::kRing * ring::rec_bytes(dv);
 }
 
+// ---- static scratch (the allocation-free entry point) ----
+// One file-scope device array serves every call of gdn_forward_static_ws in the
+// process on a given device: 24 MiB covers the ring of any supported size on a
+// device of up to 160 SMs (the largest need, d_v = 80 on 148 SMs, is 21.4 MB).
+constexpr size_t kStaticScratchBytes = 24ull << 20;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+// Address of the static scratch on the current device, looked up once per
+// device (the first call on a device must not be inside a stream capture).
+cudaError_t static_scratch(void** ptr, size_t* bytes)
+{
+    constexpr int kMaxDevices = 64;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!addr[dev]) {
+        e = cudaGetSymbolAddress(&addr[dev], g_static_scratch);
+        if (e != cudaSuccess) return e;
+    }
+    *ptr = addr[dev];
+    *bytes = kStaticScratchBytes;
+    return cudaSuccess;
+}
+
 cudaError_t launch_ring(const FwdParams& p, void* ws, size_t ws_bytes, cudaStream_t stream)
 {
     if (!ring_supported(p.dk, p.dv, ring::kC) || p.T < 1) return cudaErrorInvalidValue;

@@ -21,7 +21,7 @@ GDN_ERR_TIMEOUT = -4
 
 EXPORTS = ("gdn_forward", "gdn_state_step", "gdn_forward_f32", "gdn_state_step_f32",
            "gdn_forward_host", "gdn_workspace_bytes", "gdn_forward_ws", "gdn_state_step_ws",
-           "gdn_forward_host_ws", "gdn_status_string", "gdn_get_last_device_status",
+           "gdn_forward_host_ws", "gdn_forward_static_ws", "gdn_status_string", "gdn_get_last_device_status",
            "gdn_bf16_path", "gdn_version")
 
 
@@ -69,6 +69,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.gdn_state_step_ws.restype = I
     lib.gdn_forward_host_ws.argtypes = [P] * 15 + [I] * 7 + [P, Z, P]
     lib.gdn_forward_host_ws.restype = I
+    lib.gdn_forward_static_ws.argtypes = fwd
+    lib.gdn_forward_static_ws.restype = I
     lib.gdn_status_string.argtypes = [I]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_get_last_device_status.argtypes = [P]
@@ -197,6 +199,14 @@ def gdn_forward_host_ws(h_q, h_k, h_v, h_gate_logit, h_beta_logit, h_state_in, h
         _ptr(d_state), _ptr(d_out), B, H, T, d_k_dim, d_v_dim, frame_len, chunk_len,
         _ptr(workspace), wb, _stream(stream))
     return _check(st, "gdn_forward_host_ws", check)
+
+
+def gdn_forward_static_ws(q, k, v, gate_logit, beta_logit, state_in, state_out, out,
+                          B, H, T, d_k, d_v, frame_len, chunk_len, stream=None, check=True) -> int:
+    st = load().gdn_forward_static_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logit), _ptr(beta_logit),
+                                      _ptr(state_in), _ptr(state_out), _ptr(out),
+                                      B, H, T, d_k, d_v, frame_len, chunk_len, _stream(stream))
+    return _check(st, "gdn_forward_static_ws", check)
 
 
 def gdn_get_last_device_status(stream=None) -> int:

@@ -169,6 +169,28 @@ int gdn_forward_host_ws(const void* h_q, const void* h_k, const void* h_v,
                         int frame_len, int chunk_len, void* workspace, size_t workspace_bytes,
                         cudaStream_t stream);
 
+/*
+ * gdn_forward without a caller workspace and without any allocation: the same
+ * shared-prep ring kernel as gdn_forward_ws, its ring kept in one static device
+ * array of 24 MiB inside the library (enough for every supported size on devices
+ * of up to 160 SMs).  The pages describe no such entry point: it exists so that
+ * a caller that cannot provide memory (or must not allocate) still gets the
+ * fast path.
+ *   - Arguments, layouts and errors as gdn_forward; sizes whose ring would not
+ *     fit in the static array return GDN_ERR_UNSUPPORTED.  Sizes served without
+ *     a workspace (see gdn_workspace_bytes) run the plain path.
+ *   - The static array is looked up once per device on the first call, which
+ *     must therefore not be made inside a stream capture.
+ *   - Every call on a device uses the same array: calls that overlap in time
+ *     (other streams, other threads) race and give wrong results; order them.
+ *     Its contents persist between calls and mean nothing to the caller.
+ */
+int gdn_forward_static_ws(const void* q, const void* k, const void* v,
+                          const float* gate_logit, const float* beta_logit,
+                          const float* state_in, float* state_out, void* out,
+                          int B, int H, int T, int d_k, int d_v,
+                          int frame_len, int chunk_len, cudaStream_t stream);
+
 /* Human-readable text of a gdn_status value (static storage). */
 const char* gdn_status_string(int status);
 

@@ -148,3 +148,13 @@ def test_workspace_entry_points_validate_first():
     st = lib.gdn_forward_host_ws(A, A, A, A, A, None, None, A, A, 2 * A, 3 * A, 4 * A, 5 * A,
                                  None, 6 * A, 1, 2, 64, 112, 112, 16, 64, None, 0, None)
     assert st == G.GDN_ERR_INVALID_ARG
+
+
+def test_static_scratch_entry_validates_first():
+    lib = G.load()
+    st = lib.gdn_forward_static_ws(None, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 112, 112,
+                                   16, 64, None)
+    assert st == G.GDN_ERR_INVALID_ARG
+    st = lib.gdn_forward_static_ws(A, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 40, 112,
+                                   16, 64, None)
+    assert st == G.GDN_ERR_UNSUPPORTED

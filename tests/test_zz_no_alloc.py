@@ -1,0 +1,50 @@
+"""The allocation-free entry point gdn_forward_static_ws (the ring kept in a static
+device array inside the library) against gdn_forward_ws with a caller workspace.
+Both run the same kernel on the same inputs, so results must be identical, and stay
+so on a second call in a row (the static array keeps the previous call's contents,
+which must not matter).  Collected last on purpose: it must pass alone and after
+every other test of the session.
+"""
+
+import numpy as np
+import pytest
+
+from workloads import BLOCK, draw, long_memory, make_inputs
+
+from gpu_util import f32_device, upload
+
+pytestmark = pytest.mark.gpu
+
+
+def _cases():
+    rng = np.random.Generator(np.random.PCG64(2024))
+    return [
+        ("block, state in and out", make_inputs(BLOCK), True),
+        ("block long-memory, zero state", make_inputs(long_memory(BLOCK)), False),
+        ("40 chains, several per group of CTAs",
+         draw(rng, 2, 20, 700, 112, 112, 100, "bf16", gate_mean=0.0, gate_std=1.5, state_std=0.3), True),
+        ("d 64: a size served without a ring", draw(rng, 1, 3, 200, 64, 64, 50, "bf16", 0.0, 1.0, state_std=0.3), True),
+    ]
+
+
+@pytest.mark.parametrize("case", range(4))
+def test_static_scratch_matches_workspace_entry_two_calls(cuda, case):
+    import torch
+    import hybrid_linear_attention_frame_b200 as G
+    what, inp, with_state = _cases()[case]
+    q, k, v, g, b = upload(inp, cuda)
+    Bn, T, H, dk = inp.q.shape
+    dv = inp.v.shape[3]
+    s_in = f32_device(inp.state, cuda) if with_state else None
+    ws = G.workspace(Bn, H, T, dk, dv, 64, cuda)
+    ref_o = torch.empty_like(v)
+    ref_s = torch.empty((Bn, H, dk, dv), dtype=torch.float32, device=cuda)
+    G.gdn_forward_ws(q, k, v, g, b, s_in, ref_s, ref_o, Bn, H, T, dk, dv, inp.frame_len, 64, ws)
+    for call in range(2):
+        o = torch.full_like(v, float("nan"))
+        s = torch.full_like(ref_s, float("nan"))
+        G.gdn_forward_static_ws(q, k, v, g, b, s_in, s, o, Bn, H, T, dk, dv, inp.frame_len, 64)
+        torch.cuda.synchronize()
+        assert G.gdn_get_last_device_status() == G.GDN_OK
+        assert torch.equal(o, ref_o), f"{what}: out differs on call {call}"
+        assert torch.equal(s, ref_s), f"{what}: state differs on call {call}"
