@@ -23,6 +23,8 @@
  *   f = t / frame_len ("frame-wise").  S is d_k x d_v; row index = key dim.
  *   The decay multiplies the old state and the erase term; the new write
  *   beta k v^T is not decayed; the output reads the state after the update.
+ *   gate_mode 1 takes the other reading of "frame-wise": a_f applies once, at
+ *   the first token of frame f (t % frame_len == 0), and a_t = 1 elsewhere.
  *
  * Layouts (row-major): q,k [B,T,H,d_k]; v [B,T,H,d_v]; gate [B,ceil(T/frame_len),H];
  * beta [B,T,H]; state [B,H,d_k,d_v]; out [B,T,H,d_v].  Inputs are float32 (the
@@ -60,7 +62,7 @@ static void l2_normalise(const float* x, double* y, int n, double eps)
 static void run_chain(const float* q, const float* k, const float* v,
                       const float* gate, const float* beta, double* S, double* out,
                       int b, int h, int H, int T, int dk, int dv, int frame_len,
-                      double eps, double* work)
+                      double eps, int gate_mode, double* work)
 {
     const int F = (T + frame_len - 1) / frame_len;
     double* qn = work;
@@ -69,7 +71,8 @@ static void run_chain(const float* q, const float* k, const float* v,
     for (int t = 0; t < T; ++t) {
         const size_t row = ((size_t)b * T + t) * H + h;
         const int f = t / frame_len;
-        const double a = exp(-softplus((double)gate[((size_t)b * F + f) * H + h]));
+        const int gated = (gate_mode == 0) || (t % frame_len == 0);
+        const double a = gated ? exp(-softplus((double)gate[((size_t)b * F + f) * H + h])) : 1.0;
         const double bt = sigmoid((double)beta[row]);
         l2_normalise(q + row * dk, qn, dk, eps);
         l2_normalise(k + row * dk, kn, dk, eps);
@@ -99,16 +102,18 @@ static void run_chain(const float* q, const float* k, const float* v,
 /*
  * Run all B*H chains.  state_in may be NULL (zero initial state); state_out may
  * be NULL (final state not returned).  n_threads <= 0 lets OpenMP choose.
+ * gate_mode 0: the frame's gate at every token; 1: once, at the frame's first token.
  * Returns 0, or -1 on a bad argument or allocation failure.
  */
 int gdn_oracle_forward(const float* q, const float* k, const float* v,
                        const float* gate_logit, const float* beta_logit,
                        const float* state_in, double* state_out, double* out,
                        int B, int H, int T, int d_k, int d_v, int frame_len,
-                       double eps, int n_threads)
+                       double eps, int n_threads, int gate_mode)
 {
     if (!q || !k || !v || !gate_logit || !beta_logit || !out) return -1;
     if (B < 1 || H < 1 || T < 0 || d_k < 1 || d_v < 1 || frame_len < 1) return -1;
+    if (gate_mode != 0 && gate_mode != 1) return -1;
     const int chains = B * H;
     int failed = 0;
 #ifdef _OPENMP
@@ -129,7 +134,7 @@ int gdn_oracle_forward(const float* q, const float* k, const float* v,
         for (size_t i = 0; i < (size_t)d_k * d_v; ++i)
             S[i] = state_in ? (double)state_in[soff + i] : 0.0;
         run_chain(q, k, v, gate_logit, beta_logit, S, out, b, h, H, T, d_k, d_v,
-                  frame_len, eps, work);
+                  frame_len, eps, gate_mode, work);
         if (state_out)
             memcpy(state_out + soff, S, sizeof(double) * (size_t)d_k * d_v);
         free(S);
@@ -144,10 +149,11 @@ int gdn_oracle_forward_f64state(const float* q, const float* k, const float* v,
                                 const float* gate_logit, const float* beta_logit,
                                 const double* state_in, double* state_out, double* out,
                                 int B, int H, int T, int d_k, int d_v, int frame_len,
-                                double eps, int n_threads)
+                                double eps, int n_threads, int gate_mode)
 {
     if (!q || !k || !v || !gate_logit || !beta_logit || !out) return -1;
     if (B < 1 || H < 1 || T < 0 || d_k < 1 || d_v < 1 || frame_len < 1) return -1;
+    if (gate_mode != 0 && gate_mode != 1) return -1;
     const int chains = B * H;
     int failed = 0;
 #ifdef _OPENMP
@@ -168,7 +174,7 @@ int gdn_oracle_forward_f64state(const float* q, const float* k, const float* v,
         for (size_t i = 0; i < (size_t)d_k * d_v; ++i)
             S[i] = state_in ? state_in[soff + i] : 0.0;
         run_chain(q, k, v, gate_logit, beta_logit, S, out, b, h, H, T, d_k, d_v,
-                  frame_len, eps, work);
+                  frame_len, eps, gate_mode, work);
         if (state_out)
             memcpy(state_out + soff, S, sizeof(double) * (size_t)d_k * d_v);
         free(S);

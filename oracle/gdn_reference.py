@@ -12,7 +12,9 @@ per batch entry and head,
 
 q and k L2-normalised per token (x / sqrt(sum x^2 + eps), eps = 1e-6),
 beta_t = sigmoid(beta logit of token t), and a = exp(-softplus(gate logit of
-frame f)) shared by all tokens of latent frame f = t // frame_len.
+frame f)) shared by all tokens of latent frame f = t // frame_len.  The other
+reading of "frame-wise" (inputs with gate_mode 1) applies a_f once, at the first
+token of frame f, and a_t = 1 at the frame's other tokens.
 
 Three independent float64 forms live here:
 
@@ -69,13 +71,26 @@ def l2_normalise(x, eps=EPS):
     return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
 
 
-def token_log_gate(gate, T, frame_len):
-    """Per-token log-gate log a_t = -softplus(gate[f(t)]), f(t) = t // frame_len.
+GATE_EVERY_TOKEN = 0     # a_f at every token of frame f
+GATE_FRAME_START = 1     # a_f once, at the first token of frame f (a_t = 1 elsewhere)
 
+
+def token_log_gate(gate, T, frame_len, gate_mode=GATE_EVERY_TOKEN):
+    """Per-token log-gate log a_t, f(t) = t // frame_len.
+
+    gate_mode 0: log a_t = -softplus(gate[f(t)]) at every token ("frame-wise" read
+    as one gate shared by the frame's tokens).  gate_mode 1: the same value at the
+    first token of each frame (t % frame_len == 0) and 0 at the others ("frame-wise"
+    read as one decay per frame step).
     gate: [B, F, H]  ->  [B, T, H] float64.
     """
-    f = np.arange(T) // frame_len
-    return -softplus(np.asarray(gate, dtype=np.float64)[:, f, :])
+    t = np.arange(T)
+    la = -softplus(np.asarray(gate, dtype=np.float64)[:, t // frame_len, :])
+    if gate_mode == GATE_FRAME_START:
+        la[:, t % frame_len != 0, :] = 0.0
+    elif gate_mode != GATE_EVERY_TOKEN:
+        raise ValueError(f"unknown gate_mode {gate_mode}")
+    return la
 
 
 def _prep(inp, eps):
@@ -83,7 +98,7 @@ def _prep(inp, eps):
     qn = l2_normalise(inp.q, eps)
     kn = l2_normalise(inp.k, eps)
     v = np.asarray(inp.v, dtype=np.float64)
-    la = token_log_gate(inp.gate, T, inp.frame_len)
+    la = token_log_gate(inp.gate, T, inp.frame_len, getattr(inp, "gate_mode", GATE_EVERY_TOKEN))
     bt = sigmoid(inp.beta)
     return qn, kn, v, la, bt
 
@@ -227,7 +242,8 @@ def _load():
         lib = ctypes.CDLL(_LIB_PATH)
         fp = ctypes.POINTER(ctypes.c_float)
         dp = ctypes.POINTER(ctypes.c_double)
-        args = [fp, fp, fp, fp, fp, None, dp, dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int]
+        args = [fp, fp, fp, fp, fp, None, dp, dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int,
+                                                                          ctypes.c_int]
         f = lib.gdn_oracle_forward
         f.argtypes = args[:5] + [fp] + args[6:]
         f.restype = ctypes.c_int
@@ -260,7 +276,8 @@ def c_forward(inp, state_in=None, eps=EPS, n_threads=0, want_state=True):
     st_out_p = st_out.ctypes.data_as(dp) if want_state else ctypes.cast(None, dp)
     common = (q.ctypes.data_as(fp), k.ctypes.data_as(fp), v.ctypes.data_as(fp),
               g.ctypes.data_as(fp), b.ctypes.data_as(fp))
-    dims = (B, H, T, dk, dv, inp.frame_len, float(eps), int(n_threads))
+    dims = (B, H, T, dk, dv, inp.frame_len, float(eps), int(n_threads),
+            int(getattr(inp, "gate_mode", GATE_EVERY_TOKEN)))
     if state_in is not None and np.asarray(state_in).dtype == np.float64:
         s = np.ascontiguousarray(state_in, dtype=np.float64)
         rc = lib.gdn_oracle_forward_f64state(*common, s.ctypes.data_as(dp), st_out_p,

@@ -50,6 +50,9 @@ class Inputs:
     state: Optional[np.ndarray]
     io_dtype: str
     frame_len: int
+    # where the frame's gate applies: 0 = at every token of the frame, 1 = once, at
+    # the frame's first token (the two readings of "frame-wise"; see the oracle)
+    gate_mode: int = 0
 
     @property
     def shape(self):
