@@ -56,6 +56,9 @@ def parse_args(argv=None):
                     help="target wall time of the oracle sample")
     ap.add_argument("--profile-tokens", type=int, default=0,
                     help="profiling case: two layer calls on the layer's first T tokens, no timing")
+    ap.add_argument("--gate-mode", choices=["token", "frame"], default="token",
+                    help="token: a frame's gate at each of its tokens (gdn_forward*); frame: once, at "
+                         "the frame's first token (gdn_forward_gated, gate_mode 1)")
     ap.add_argument("--path", choices=["ws", "plain"], default="ws",
                     help="ws: gdn_forward_ws (shared prep through a workspace ring); "
                          "plain: gdn_forward (no workspace)")
@@ -332,13 +335,18 @@ def run_ours(args, w, rank, world, local):
     ws = G.workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.chunk_len, device) if use_ws else None
     ws_args = (ws.data_ptr(), ws.numel()) if use_ws else (None, 0)
 
+    gate_mode = 1 if args.gate_mode == "frame" else 0
+
     def layer_call():
-        if use_ws:
+        if gate_mode:
+            st = lib.gdn_forward_gated(*ptrs, *dims, gate_mode, *ws_args, sptr)
+        elif use_ws:
             st = lib.gdn_forward_ws(*ptrs, *dims, *ws_args, sptr)
         else:
             st = lib.gdn_forward(*ptrs, *dims, sptr)
         if st != 0:
-            raise G.GdnError(st, "gdn_forward_ws" if use_ws else "gdn_forward")
+            raise G.GdnError(st, "gdn_forward_gated" if gate_mode else
+                             ("gdn_forward_ws" if use_ws else "gdn_forward"))
 
     for _ in range(args.warmup):
         for _ in range(layers):
@@ -415,9 +423,13 @@ def run_ours(args, w, rank, world, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": dict(workload_config(w, layers),
-                           api=("gdn_forward_ws (C ABI, device buffers, workspace "
+                           gate_placement=("once per frame, at its first token (gate_mode 1)" if gate_mode
+                                           else "at every token of the frame"),
+                           api=(("gdn_forward_gated" if gate_mode else "gdn_forward_ws") +
+                                " (C ABI, device buffers, workspace "
                                 f"{ws.numel() / 2**20:.1f} MiB reused by every layer)") if use_ws
-                           else "gdn_forward (C ABI, device buffers)"),
+                           else ("gdn_forward_gated" if gate_mode else "gdn_forward") +
+                           " (C ABI, device buffers)"),
             "roofline": roofline,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * layers,
             "clocks": clock_rec}

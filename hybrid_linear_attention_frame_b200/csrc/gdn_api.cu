@@ -78,6 +78,7 @@ int validate(const void* q, const void* k, const void* v, const float* gate,
     p->out = const_cast<void*>(out);
     p->B = B; p->H = H; p->T = T; p->dk = dk; p->dv = dv; p->frame_len = frame_len;
     p->F = (int)F;
+    p->gate_mode = 0;
     return GDN_OK;
 }
 
@@ -247,6 +248,37 @@ int gdn_forward_host_ws(const void* h_q, const void* h_k, const void* h_v,
     return forward_host(h_q, h_k, h_v, h_gate_logit, h_beta_logit, h_state_in, h_state_out, h_out, d_q, d_k,
                         d_v, d_gate_logit, d_beta_logit, d_state, d_out, B, H, T, d_k_dim, d_v_dim, frame_len,
                         chunk_len, workspace, workspace_bytes, stream);
+}
+
+int gdn_forward_gated(const void* q, const void* k, const void* v,
+                      const float* gate_logit, const float* beta_logit,
+                      const float* state_in, float* state_out, void* out,
+                      int B, int H, int T, int d_k, int d_v, int frame_len, int chunk_len,
+                      int gate_mode, void* workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (gate_mode != 0 && gate_mode != 1) return GDN_ERR_INVALID_ARG;
+    gdn::FwdParams p;
+    int st = validate(q, k, v, gate_logit, beta_logit, state_in, state_out, out, true, 2,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
+    if (st != GDN_OK) return st;
+    p.gate_mode = gate_mode;
+    return workspace ? run_bf16_ws(p, chunk_len, workspace, workspace_bytes, stream)
+                     : run_bf16(p, chunk_len, stream);
+}
+
+int gdn_forward_gated_f32(const float* q, const float* k, const float* v,
+                          const float* gate_logit, const float* beta_logit,
+                          const float* state_in, float* state_out, float* out,
+                          int B, int H, int T, int d_k, int d_v, int frame_len, int chunk_len,
+                          int gate_mode, cudaStream_t stream)
+{
+    if (gate_mode != 0 && gate_mode != 1) return GDN_ERR_INVALID_ARG;
+    gdn::FwdParams p;
+    int st = validate(q, k, v, gate_logit, beta_logit, state_in, state_out, out, true, 4,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
+    if (st != GDN_OK) return st;
+    p.gate_mode = gate_mode;
+    return to_status(gdn::launch_ffma<float>(p, chunk_len, stream));
 }
 
 int gdn_forward_static_ws(const void* q, const void* k, const void* v,

@@ -34,7 +34,15 @@ struct FwdParams {
     float* state_out;        // [B, H, dk, dv] or null
     void* out;               // [B, T, H, dv] or null
     int B, H, T, dk, dv, frame_len, F;
+    int gate_mode;           // 0: a frame's gate at each of its tokens; 1: once, at its first token
 };
+
+// Does token t of the call take its frame's gate?  Frame f covers tokens
+// f*frame_len .. (f+1)*frame_len - 1; gate_mode 0 applies a_f at all of them,
+// gate_mode 1 only at the first (the two readings of "frame-wise").
+__device__ __forceinline__ bool gate_applies(const FwdParams& p, int t) {
+    return p.gate_mode == 0 || (t % p.frame_len) == 0;
+}
 
 __device__ __forceinline__ float softplus_f(float x) {
     // log(1 + e^x) = max(x, 0) + log1p(e^{-|x|})

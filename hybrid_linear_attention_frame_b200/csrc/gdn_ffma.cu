@@ -92,7 +92,7 @@ chunk_ffma_kernel(FwdParams p)
             if (tid < L) {
                 const int t = c0 + tid;
                 const float g = p.gate[((size_t)b * p.F + t / p.frame_len) * p.H + h];
-                la = -softplus_f(g);
+                la = gate_applies(p, t) ? -softplus_f(g) : 0.0f;
                 bt = sigmoid_f(p.beta[((size_t)b * p.T + t) * p.H + h]);
             }
             Gs[tid] = la;   // log-gate for now; prefix sum below

@@ -325,8 +325,8 @@ __device__ __noinline__ void prep_gates_tables(const FwdParams& p, const Item& j
             g1 = __ldg(p.gate + ((size_t)jt.b * p.F + (t0 + 1) / p.frame_len) * p.H + jt.h);
             r1 = __ldg(p.beta + ((size_t)jt.b * p.T + t0 + 1) * p.H + jt.h);
         }
-        const float la0 = (i0 < L) ? -softplus_fast(g0) : 0.0f;
-        const float la1 = (i1 < L) ? -softplus_fast(g1) : 0.0f;
+        const float la0 = (i0 < L && gate_applies(p, t0)) ? -softplus_fast(g0) : 0.0f;
+        const float la1 = (i1 < L && gate_applies(p, t0 + 1)) ? -softplus_fast(g1) : 0.0f;
         float x = la0 + la1;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {

@@ -454,8 +454,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int i0 = 2 * lane, i1 = i0 + 1;
                 const float g0 = pg0, g1 = pg1, r0 = pb0, r1 = pb1;
                 if (cc + 1 < ntk) load_logits(cc + 1, pg0, pg1, pb0, pb1);
-                const float la0 = (i0 < L) ? -softplus_fast(g0) : 0.0f;
-                const float la1 = (i1 < L) ? -softplus_fast(g1) : 0.0f;
+                const float la0 = (i0 < L && gate_applies(p, cc * kC + i0)) ? -softplus_fast(g0) : 0.0f;
+                const float la1 = (i1 < L && gate_applies(p, cc * kC + i1)) ? -softplus_fast(g1) : 0.0f;
                 float x = la0 + la1;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {

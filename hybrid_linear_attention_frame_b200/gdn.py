@@ -21,7 +21,8 @@ GDN_ERR_TIMEOUT = -4
 
 EXPORTS = ("gdn_forward", "gdn_state_step", "gdn_forward_f32", "gdn_state_step_f32",
            "gdn_forward_host", "gdn_workspace_bytes", "gdn_forward_ws", "gdn_state_step_ws",
-           "gdn_forward_host_ws", "gdn_forward_static_ws", "gdn_status_string", "gdn_get_last_device_status",
+           "gdn_forward_host_ws", "gdn_forward_static_ws", "gdn_forward_gated",
+           "gdn_forward_gated_f32", "gdn_status_string", "gdn_get_last_device_status",
            "gdn_bf16_path", "gdn_version")
 
 
@@ -71,6 +72,10 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.gdn_forward_host_ws.restype = I
     lib.gdn_forward_static_ws.argtypes = fwd
     lib.gdn_forward_static_ws.restype = I
+    lib.gdn_forward_gated.argtypes = [P] * 8 + [I] * 8 + [P, Z, P]
+    lib.gdn_forward_gated.restype = I
+    lib.gdn_forward_gated_f32.argtypes = [P] * 8 + [I] * 8 + [P]
+    lib.gdn_forward_gated_f32.restype = I
     lib.gdn_status_string.argtypes = [I]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_get_last_device_status.argtypes = [P]
@@ -207,6 +212,31 @@ def gdn_forward_static_ws(q, k, v, gate_logit, beta_logit, state_in, state_out, 
                                       _ptr(state_in), _ptr(state_out), _ptr(out),
                                       B, H, T, d_k, d_v, frame_len, chunk_len, _stream(stream))
     return _check(st, "gdn_forward_static_ws", check)
+
+
+GATE_EVERY_TOKEN = 0
+GATE_FRAME_START = 1
+
+
+def gdn_forward_gated(q, k, v, gate_logit, beta_logit, state_in, state_out, out,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, gate_mode, workspace=None,
+                      workspace_bytes=None, stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().gdn_forward_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logit), _ptr(beta_logit),
+                                  _ptr(state_in), _ptr(state_out), _ptr(out),
+                                  B, H, T, d_k, d_v, frame_len, chunk_len, gate_mode,
+                                  _ptr(workspace), wb, _stream(stream))
+    return _check(st, "gdn_forward_gated", check)
+
+
+def gdn_forward_gated_f32(q, k, v, gate_logit, beta_logit, state_in, state_out, out,
+                          B, H, T, d_k, d_v, frame_len, chunk_len, gate_mode, stream=None,
+                          check=True) -> int:
+    st = load().gdn_forward_gated_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logit), _ptr(beta_logit),
+                                      _ptr(state_in), _ptr(state_out), _ptr(out),
+                                      B, H, T, d_k, d_v, frame_len, chunk_len, gate_mode,
+                                      _stream(stream))
+    return _check(st, "gdn_forward_gated_f32", check)
 
 
 def gdn_get_last_device_status(stream=None) -> int:

@@ -191,6 +191,32 @@ int gdn_forward_static_ws(const void* q, const void* k, const void* v,
                           int B, int H, int T, int d_k, int d_v,
                           int frame_len, int chunk_len, cudaStream_t stream);
 
+/*
+ * The other reading of "frame-wise" (gate placement).  gdn_forward applies a
+ * frame's gate a_f = exp(-softplus(gate_logit[f])) at every token of frame f
+ * (gate_mode 0).  With gate_mode 1 it applies a_f once, at the first token of
+ * frame f (t % frame_len == 0; a_t = 1 at the frame's other tokens), i.e. one
+ * decay per latent-frame step.  The pages name the layer "frame-wise Gated
+ * DeltaNet" (sglang cookbook SANA-WM page, section 1 architecture table) without
+ * fixing which; both are offered.
+ *   gdn_forward_gated: bf16 as gdn_forward, or as gdn_forward_ws when
+ *     `workspace` is not NULL (then sized by gdn_workspace_bytes).
+ *   gdn_forward_gated_f32: float32 reference mode as gdn_forward_f32.
+ * gate_mode outside {0, 1} gives GDN_ERR_INVALID_ARG; everything else as the
+ * entry points named.
+ */
+int gdn_forward_gated(const void* q, const void* k, const void* v,
+                      const float* gate_logit, const float* beta_logit,
+                      const float* state_in, float* state_out, void* out,
+                      int B, int H, int T, int d_k, int d_v, int frame_len, int chunk_len,
+                      int gate_mode, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+int gdn_forward_gated_f32(const float* q, const float* k, const float* v,
+                          const float* gate_logit, const float* beta_logit,
+                          const float* state_in, float* state_out, float* out,
+                          int B, int H, int T, int d_k, int d_v, int frame_len, int chunk_len,
+                          int gate_mode, cudaStream_t stream);
+
 /* Human-readable text of a gdn_status value (static storage). */
 const char* gdn_status_string(int status);
 

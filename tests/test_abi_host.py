@@ -158,3 +158,16 @@ def test_static_scratch_entry_validates_first():
     st = lib.gdn_forward_static_ws(A, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 40, 112,
                                    16, 64, None)
     assert st == G.GDN_ERR_UNSUPPORTED
+
+
+def test_gated_entry_points_validate_gate_mode():
+    lib = G.load()
+    st = lib.gdn_forward_gated(A, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 32, 32, 16, 16,
+                               2, None, 0, None)
+    assert st == G.GDN_ERR_INVALID_ARG
+    st = lib.gdn_forward_gated_f32(A, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 32, 32, 16, 16,
+                                   -1, None)
+    assert st == G.GDN_ERR_INVALID_ARG
+    st = lib.gdn_forward_gated(None, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 32, 32, 16, 16,
+                               1, None, 0, None)
+    assert st == G.GDN_ERR_INVALID_ARG
