@@ -17,12 +17,14 @@
 // chunk's record (W and P as ready-made 128-byte-swizzled operand images, U in
 // 16-column slices, the per-token scalars) into ring slot n mod kRing and then
 // publishes it with a GPU-scope release store.  Every CTA of the group runs the
-// chain for its own 16 columns over all chunks: a loader warp acquires the
-// record, pulls it into shared memory with bulk copies (plus the chunk's q and
-// k tiles by TMA) and reports the slot consumed once the chain is done with it
-// (the loader publishes that, so that the chain warps never wait on a fence).
-// A producer re-fills a slot only after every CTA of the group has consumed
-// it.  Each wait depends only on chunks with a smaller index, and the launch is
+// chain for its own 16 columns over all chunks, from two shared-memory slots,
+// each filled in two parts: loader A acquires the ready flags and copies part A
+// (the chunk's q tiles by TMA, the W image by bulk copy) as soon as MMA1 two
+// chunks back has read the slot; loader B copies part B (k tiles, P, the U
+// slice, the scalars) once the chunk two back is done with entirely, then
+// reports the ring slot consumed (so the chain warps never wait on a fence).
+// A producer re-fills a ring slot only after every CTA of the group has
+// consumed it.  Each wait depends only on chunks with a smaller index, and the launch is
 // cooperative (all CTAs resident), so the protocol cannot deadlock; every wait
 // is bounded all the same and gives up with GDN_ERR_TIMEOUT.
 //
