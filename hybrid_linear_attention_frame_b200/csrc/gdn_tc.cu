@@ -285,9 +285,8 @@ __device__ __forceinline__ void tile16x8(float (&d)[4], XF X, YF Y, int lane) {
 // Every output 8-column tile of a combination depends on the same columns of
 // the intermediate product only, so each warp owns whole column tiles and
 // keeps its intermediate in a private scratch (MSw: [32][8] per warp).
-// Run by the 128 solve threads (st = 0..127, warp pw = st / 32), which share the
-// named barrier `bar_id`.
-__device__ void unit_lower_inverse_64(float* AXI, float* MS, int st, uint32_t bar_id = kBarSolve) {
+// Run by the 128 solve threads (st = 0..127, warp pw = st / 32).
+__device__ void unit_lower_inverse_64(float* AXI, float* MS, int st) {
     const int pw = st >> 5, lane = st & 31, g = lane >> 2, t = lane & 3;
     if (st < 64) {
         // column j of the inverse of diagonal block o: right-looking substitution, so
@@ -304,7 +303,7 @@ __device__ void unit_lower_inverse_64(float* AXI, float* MS, int st, uint32_t ba
         for (int i = 0; i < 16; ++i)
             if (i >= j) AXI[(o + i) * kXS + o + j] = x[i];
     }
-    named_bar_sync(bar_id, kSolveThreads);
+    named_bar_sync(kBarSolve, kSolveThreads);
     float* MSw = MS + pw * 32 * kMS;
     // level 1: blocks (1,0) and (3,2): Y = -D_hi^{-1} (A_{hi,lo} D_lo^{-1}); warp -> (pair, 8 columns)
     {
@@ -326,7 +325,7 @@ __device__ void unit_lower_inverse_64(float* AXI, float* MS, int st, uint32_t ba
         AXI[(hi + g + 8) * kXS + lo + n0 + 2 * t] = -y[2];
         AXI[(hi + g + 8) * kXS + lo + n0 + 2 * t + 1] = -y[3];
     }
-    named_bar_sync(bar_id, kSolveThreads);
+    named_bar_sync(kBarSolve, kSolveThreads);
     // level 2: block rows 32-63, columns 0-31; warp -> 8 columns
     {
         const int n0 = 8 * pw;
@@ -353,7 +352,7 @@ __device__ void unit_lower_inverse_64(float* AXI, float* MS, int st, uint32_t ba
             AXI[(r0 + 8) * kXS + n0 + 2 * t + 1] = -y[3];
         }
     }
-    named_bar_sync(bar_id, kSolveThreads);
+    named_bar_sync(kBarSolve, kSolveThreads);
 }
 
 // ---------------------------------------------------------------- the kernel
