@@ -19,6 +19,7 @@ size_t ring_workspace_bytes(int G, int dv);
 cudaError_t launch_ring(const FwdParams& p, void* ws, size_t ws_bytes, cudaStream_t stream);
 cudaError_t static_scratch(void** ptr, size_t* bytes);
 int read_and_clear_device_status(cudaStream_t stream);
+void set_wait_limit_ns(uint64_t ns);
 }  // namespace gdn
 
 namespace {
@@ -357,6 +358,12 @@ const char* gdn_status_string(int status)
 int gdn_get_last_device_status(cudaStream_t stream)
 {
     return gdn::read_and_clear_device_status(stream);
+}
+
+int gdn_set_wait_limit_ns(unsigned long long ns)
+{
+    gdn::set_wait_limit_ns((uint64_t)ns);
+    return GDN_OK;
 }
 
 int gdn_bf16_path(int d_k, int d_v, int chunk_len)

@@ -303,14 +303,6 @@ __device__ __forceinline__ void item_advance(Item& it, const FwdParams& p, int G
 }
 
 
-// Bounded wait used only on the way out after an abort (async copies or MMAs
-// that may still be in flight must land before shared memory and TMEM go).
-__device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < limit_ns) {
-    }
-}
-
 // Gates (G, beta) and decay tables of chunk jt into `scx`, run by the 128 prep
 // threads of warps pw 4-7 (out of line: it has two call sites).
 __device__ __noinline__ void prep_gates_tables(const FwdParams& p, const Item& jt, float* scx, int pw, int lane,
@@ -568,8 +560,8 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!ok && pending >= 0) {
             // MMAs possibly still in flight must finish before TMEM is released
-            drain_wait(bar((uint32_t)pending), 0, lim);
-            drain_wait(bar((uint32_t)pending), 1, lim);
+            drain_wait(bar((uint32_t)pending), 0);
+            drain_wait(bar((uint32_t)pending), 1);
         }
     } else if (warp < 12) {
         // ======================= prep (warps 4-11) =======================
@@ -821,8 +813,8 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!ok) {
             if (pw == 4) {
-                if (ptma_issued > ptma_waited) drain_wait(bar(kBarPTma), (uint32_t)((ptma_issued - 1) & 1), lim);
-                if (mma_pending >= 0) drain_wait(bar((uint32_t)mma_pending), (uint32_t)(m & 1), lim);
+                if (ptma_issued > ptma_waited) drain_wait(bar(kBarPTma), (uint32_t)((ptma_issued - 1) & 1));
+                if (mma_pending >= 0) drain_wait(bar((uint32_t)mma_pending), (uint32_t)(m & 1));
             }
         }
     } else if (warp < kLoaderA) {
@@ -870,8 +862,8 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (lane == 0) mbar_arrive(bar(kBarFreeB + s));   // P, E and this chunk's TMEM are done with
         }
         if (!ok && m2p_pending && warp == kOutWarp0) {
-            drain_wait(bar(kBarM2P), 0, lim);
-            drain_wait(bar(kBarM2P), 1, lim);
+            drain_wait(bar(kBarM2P), 0);
+            drain_wait(bar(kBarM2P), 1);
         }
     } else if (warp == kLoaderA) {
         // ======================= loader A (warp 14): q and W tiles =======================
@@ -923,7 +915,7 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!ok && lane == 0) {
             // copies still in flight must land before shared memory goes away
             for (int n = max(0, issued - 2); n < issued; ++n)
-                drain_wait(bar(kBarFullA + (n & 1)), (uint32_t)((n >> 1) & 1), lim);
+                drain_wait(bar(kBarFullA + (n & 1)), (uint32_t)((n >> 1) & 1));
         }
         __syncwarp();
     } else {
@@ -960,7 +952,7 @@ gdn_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!ok && lane == 0) {
             for (int n = max(0, issued - 2); n < issued; ++n)
-                drain_wait(bar(kBarFullB + (n & 1)), (uint32_t)((n >> 1) & 1), lim);
+                drain_wait(bar(kBarFullB + (n & 1)), (uint32_t)((n >> 1) & 1));
         }
         __syncwarp();
     }

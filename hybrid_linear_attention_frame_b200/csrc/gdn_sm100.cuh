@@ -76,6 +76,7 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
     return ok != 0;
 }
 
+
 // Wait for the phase with the given parity to complete, giving up after
 // `limit_ns` nanoseconds or as soon as another thread has raised `*abort`.
 // On giving up it raises *abort, records `code` in the device status word
@@ -102,6 +103,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           uint64_t limit_ns, int code) {
     if (mbar_try_wait(bar, parity)) return true;
     return mbar_wait_slow(bar, parity, abort, limit_ns, code);
+}
+
+// Waits on the way out after an abort, for async copies or MMAs still in flight
+// (they must land before shared memory and TMEM are released).  Their bound is
+// fixed, independent of the configurable wait limit: in-flight work completes
+// within microseconds, and cutting these waits short would be unsafe.
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
+
+__device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kDrainLimitNs) {
+    }
 }
 
 // ---------------------------------------------------------------- fences and named barriers

@@ -505,6 +505,8 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         };
         if (ntk > 0) compute_gates(0);
+        int mma_bar = -1;                     // MMA group issued and not yet waited for
+        uint32_t mma_par = 0;
         int c = 0;
         for (; c < ntk; ++c) {
             const int s = c & 1;
@@ -518,9 +520,12 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 issue_m1(slot, sbt, tmem, nks);
                 mma_commit_warp(bar(kBarM1));
             }
+            mma_bar = kBarM1;
+            mma_par = (uint32_t)(c & 1);
             if (c > 0) output(c - 1);          // previous chunk's output while MMA1 runs
             ok = mbar_wait(bar(kBarM1), (uint32_t)(c & 1), abort_flag, lim, 4);
             if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
+            mma_bar = -1;
             tc_fence_after();
             {
                 float v[16];
@@ -554,8 +559,11 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 issue_m2(slot, base, ebt, ept, tmem, s);
                 mma_commit_warp(bar(kBarM2));
             }
+            mma_bar = kBarM2;
+            mma_par = (uint32_t)(c & 1);
             ok = mbar_wait(bar(kBarM2), (uint32_t)(c & 1), abort_flag, lim, 5);
             if (!group_all(kBarChain, kChainThreads, ok)) { ok = false; break; }
+            mma_bar = -1;
             tc_fence_after();
             {
                 const int m = tid;
@@ -582,14 +590,12 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         if (ok && ntk > 0) output(ntk - 1);
         if (!ok && warp == 0) {
-            // drain tile loads still in flight before the shared memory goes away (bounded)
+            // drain tile loads and an MMA group still in flight before the shared memory
+            // and TMEM go away (bounded)
             if (elect_one()) {
-                for (int cc = max(0, tma_issued - kSlots); cc < tma_issued; ++cc) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait(bar(kBarTma + cc % kSlots), (uint32_t)((cc / kSlots) & 1)) &&
-                           globaltimer_ns() - t0 < lim) {
-                    }
-                }
+                if (mma_bar >= 0) drain_wait(bar((uint32_t)mma_bar), mma_par);
+                for (int cc = max(0, tma_issued - kSlots); cc < tma_issued; ++cc)
+                    drain_wait(bar(kBarTma + cc % kSlots), (uint32_t)((cc / kSlots) & 1));
             }
             __syncwarp();
         }
@@ -614,7 +620,12 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             return got;
         };
         bool pre_ok = true;
-        if (pw == 4 && ntk > 0) pre_ok = prefetch_g1(0);
+        int g1_issued = 0, g1_waited = 0;     // chunks whose Gram MMAs were issued / waited for
+        int wu_chunk = -1;                    // chunk whose W/U MMAs were issued and not waited for
+        if (pw == 4 && ntk > 0) {
+            pre_ok = prefetch_g1(0);
+            g1_issued = pre_ok ? 1 : 0;
+        }
         for (int c = 0; c < ntk; ++c) {
             const int s = c & 1, gbuf = c & 1;
             const uint32_t slot = base + (uint32_t)(c % kSlots) * kSlotBytes;
@@ -623,6 +634,7 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ok = ok && mbar_wait(bar(kBarTma + (c % kSlots)), (uint32_t)((c / kSlots) & 1), abort_flag, lim, 1);
             ok = ok && mbar_wait(bar(kBarG1 + gbuf), (uint32_t)((c >> 1) & 1), abort_flag, lim, 2);
             if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            g1_waited = c + 1;
             tc_fence_after();
             const uint32_t tg = tmem + kColG + 128u * gbuf;
             // ---- norms from the Gram diagonal: |k_i|^2 (lanes 0-63), |q_i|^2 (lanes 64-127) ----
@@ -700,7 +712,10 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             bool ok2 = true;
             if (pw == 4) {
                 // next chunk's Gram matrices run on the tensor cores during this chunk's solve
-                if (c + 1 < ntk) ok2 = prefetch_g1(c + 1);
+                if (c + 1 < ntk) {
+                    ok2 = prefetch_g1(c + 1);
+                    if (ok2) g1_issued = c + 2;
+                }
             } else if (pw < 4) {
                 // ---- T = (I + A)^{-1} diag(beta), T' = T diag(e^G / |k|) ----
                 unit_lower_inverse_64(AXI, MSf, pt);
@@ -737,8 +752,10 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 issue_wu(slot, base, tmem, dk, s);
                 mma_commit_warp(bar(kBarWU));
             }
+            wu_chunk = c;
             ok = mbar_wait(bar(kBarWU), (uint32_t)(c & 1), abort_flag, lim, 3);
             if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            wu_chunk = -1;
             tc_fence_after();
             // ---- W (TMEM lanes 0-63) to smem next to Q ----
             if (qtr < 2) {
@@ -758,13 +775,13 @@ gdn_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             named_bar_sync(kBarPrep, kPrepThreads);
             if (pt == 0) mbar_arrive(bar(kBarReady + s));
         }
-        if (!ok && pw == 4) {
-            // a Gram MMA may still be in flight: wait for it (bounded) before TMEM is freed
-            const uint64_t t0 = globaltimer_ns();
-            for (int bb = 0; bb < 2; ++bb)
-                while (!mbar_try_wait(bar(kBarG1 + bb), 0) && !mbar_try_wait(bar(kBarG1 + bb), 1) &&
-                       globaltimer_ns() - t0 < lim) {
-                }
+        if (!ok) {
+            // Gram MMAs issued and not waited for (chunk cc on buffer cc & 1, its (cc >> 1)-th
+            // use), and the W/U group if its wait gave up, must finish before TMEM is freed
+            if (pw == 4)
+                for (int cc = g1_waited; cc < g1_issued; ++cc)
+                    drain_wait(bar(kBarG1 + (cc & 1)), (uint32_t)((cc >> 1) & 1));
+            if (pw == 0 && wu_chunk >= 0) drain_wait(bar(kBarWU), (uint32_t)(wu_chunk & 1));
         }
     }
 
@@ -811,9 +828,13 @@ bool make_map(CUtensorMap* map, const void* base, int inner, int H, int T, int B
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-uint64_t g_wait_limit_ns = 2000000000ull;   // 2 s
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // 2 s
+uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 
 }  // namespace
+
+// Bound of every device-side wait of later launches (0 restores the default).
+void set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns ? ns : kDefaultWaitLimitNs; }
 
 bool tc_supported(int dk, int dv, int chunk_len)
 {

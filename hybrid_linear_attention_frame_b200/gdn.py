@@ -22,7 +22,7 @@ GDN_ERR_TIMEOUT = -4
 EXPORTS = ("gdn_forward", "gdn_state_step", "gdn_forward_f32", "gdn_state_step_f32",
            "gdn_forward_host", "gdn_workspace_bytes", "gdn_forward_ws", "gdn_state_step_ws",
            "gdn_forward_host_ws", "gdn_forward_static_ws", "gdn_forward_gated",
-           "gdn_forward_gated_f32", "gdn_status_string", "gdn_get_last_device_status",
+           "gdn_forward_gated_f32", "gdn_set_wait_limit_ns", "gdn_status_string", "gdn_get_last_device_status",
            "gdn_bf16_path", "gdn_version")
 
 
@@ -78,6 +78,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.gdn_forward_gated_f32.restype = I
     lib.gdn_status_string.argtypes = [I]
     lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.gdn_set_wait_limit_ns.restype = I
     lib.gdn_get_last_device_status.argtypes = [P]
     lib.gdn_get_last_device_status.restype = I
     lib.gdn_bf16_path.argtypes = [I, I, I]
@@ -237,6 +239,10 @@ def gdn_forward_gated_f32(q, k, v, gate_logit, beta_logit, state_in, state_out, 
                                       B, H, T, d_k, d_v, frame_len, chunk_len, gate_mode,
                                       _stream(stream))
     return _check(st, "gdn_forward_gated_f32", check)
+
+
+def gdn_set_wait_limit_ns(ns: int) -> int:
+    return load().gdn_set_wait_limit_ns(int(ns))
 
 
 def gdn_get_last_device_status(stream=None) -> int:

@@ -229,6 +229,16 @@ const char* gdn_status_string(int status);
  */
 int gdn_get_last_device_status(cudaStream_t stream);
 
+/*
+ * Bound, in nanoseconds, of every device-side wait of the launches that follow
+ * (process-wide; default 2 s; 0 restores the default).  A bound below what a call
+ * legitimately needs makes it give up: the kernel stops its work, leaves its
+ * outputs undefined and records GDN_ERR_TIMEOUT for gdn_get_last_device_status;
+ * the context stays usable.  Meant for testing that path.  Waits for work that is
+ * already in flight when a kernel gives up keep a fixed 2 s bound.  Returns GDN_OK.
+ */
+int gdn_set_wait_limit_ns(unsigned long long ns);
+
 /* Which kernel the bf16 entry points dispatch to for the given sizes
  * (0 = FFMA chunked kernel, 1 = tensor-core chunked kernel). */
 int gdn_bf16_path(int d_k, int d_v, int chunk_len);

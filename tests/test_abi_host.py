@@ -171,3 +171,9 @@ def test_gated_entry_points_validate_gate_mode():
     st = lib.gdn_forward_gated(None, 2 * A, 3 * A, 4 * A, 5 * A, None, None, 6 * A, 1, 2, 64, 32, 32, 16, 16,
                                1, None, 0, None)
     assert st == G.GDN_ERR_INVALID_ARG
+
+
+def test_wait_limit_setter_needs_no_device():
+    # sets a process-wide host value read at the next launch; 0 restores the default
+    assert G.gdn_set_wait_limit_ns(1000) == G.GDN_OK
+    assert G.gdn_set_wait_limit_ns(0) == G.GDN_OK
