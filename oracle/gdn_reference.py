@@ -35,6 +35,18 @@ Three independent float64 forms live here:
 
 and a ctypes wrapper, ``c_forward``, for the C token recurrence in
 ``gdn_oracle.c`` (OpenMP over chains), used at full sizes.
+
+The dense checkpoint's bidirectional GDN (sglang cookbook SANA-WM page,
+dense-bidirectional section) is not defined on the pages; it is fixed here as
+the sum of the forward scan and the same rule run from the last token to the
+first, both from a zero state, every token keeping its own q, k, v, beta and the
+gate of its own frame (at every token):
+
+    R_t = a_t (I - beta_t k_t k_t^T) R_{t+1} + beta_t k_t v_t^T,  R_T = 0,
+    o_t = S_t^T q_t + R_t^T q_t.
+
+``token_recurrence_backward`` is that backward loop, ``bidirectional`` the sum,
+``c_bidirectional`` the C form of the sum.
 """
 
 import ctypes
@@ -139,6 +151,33 @@ def token_recurrence(inp, state_in=None, eps=EPS, return_states=False):
     if return_states:
         return out, S, np.stack(states) if states else np.zeros((0,) + S.shape)
     return out, S
+
+
+def token_recurrence_backward(inp, eps=EPS):
+    """The same rule run from the last token to the first, from a zero state:
+    R_t = a_t (I - beta_t k_t k_t^T) R_{t+1} + beta_t k_t v_t^T, output R_t^T q_t.
+    Token t keeps its own frame's gate.  Returns out [B,T,H,d_v]."""
+    if getattr(inp, "gate_mode", GATE_EVERY_TOKEN) != GATE_EVERY_TOKEN:
+        raise ValueError("the backward scan takes the gate at every token only")
+    qn, kn, v, la, bt = _prep(inp, eps)
+    B, T, H, dk = qn.shape
+    R = np.zeros((B, H, dk, v.shape[3]))
+    out = np.zeros(v.shape)
+    for t in range(T - 1, -1, -1):
+        a = np.exp(la[:, t, :])[:, :, None, None]
+        b = bt[:, t, :][:, :, None, None]
+        k_t = kn[:, t, :, :]
+        kR = np.einsum("bhi,bhij->bhj", k_t, R)              # k^T R_{t+1}
+        R = a * (R - b * k_t[..., :, None] * kR[..., None, :]) \
+            + b * k_t[..., :, None] * v[:, t, :, :][..., None, :]
+        out[:, t] = np.einsum("bhij,bhi->bhj", R, qn[:, t])
+    return out
+
+
+def bidirectional(inp, eps=EPS):
+    """Forward scan plus backward scan, both from a zero state.  Returns out [B,T,H,d_v]."""
+    fwd, _ = token_recurrence(inp, None, eps)
+    return fwd + token_recurrence_backward(inp, eps)
 
 
 # ----------------------------------------------------------------------------
@@ -250,6 +289,9 @@ def _load():
         g = lib.gdn_oracle_forward_f64state
         g.argtypes = args[:5] + [dp] + args[6:]
         g.restype = ctypes.c_int
+        h = lib.gdn_oracle_bidirectional
+        h.argtypes = [fp] * 5 + [dp] + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int]
+        h.restype = ctypes.c_int
         lib.gdn_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -289,3 +331,26 @@ def c_forward(inp, state_in=None, eps=EPS, n_threads=0, want_state=True):
     if rc != 0:
         raise RuntimeError("gdn_oracle_forward failed")
     return out, st_out
+
+
+def c_bidirectional(inp, eps=EPS, n_threads=0):
+    """C form of ``bidirectional`` (forward plus backward scan from zero states)."""
+    if getattr(inp, "gate_mode", GATE_EVERY_TOKEN) != GATE_EVERY_TOKEN:
+        raise ValueError("the bidirectional form takes the gate at every token only")
+    lib = _load()
+    B, T, H, dk = inp.q.shape
+    dv = inp.v.shape[3]
+    fp = ctypes.POINTER(ctypes.c_float)
+    dp = ctypes.POINTER(ctypes.c_double)
+
+    def f32(a):
+        return np.ascontiguousarray(a, dtype=np.float32)
+
+    q, k, v, g, b = f32(inp.q), f32(inp.k), f32(inp.v), f32(inp.gate), f32(inp.beta)
+    out = np.empty((B, T, H, dv), dtype=np.float64)
+    rc = lib.gdn_oracle_bidirectional(q.ctypes.data_as(fp), k.ctypes.data_as(fp), v.ctypes.data_as(fp),
+                                      g.ctypes.data_as(fp), b.ctypes.data_as(fp), out.ctypes.data_as(dp),
+                                      B, H, T, dk, dv, inp.frame_len, float(eps), int(n_threads))
+    if rc != 0:
+        raise RuntimeError("gdn_oracle_bidirectional failed")
+    return out
