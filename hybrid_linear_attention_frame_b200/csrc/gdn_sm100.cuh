@@ -86,11 +86,9 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
                                             uint64_t limit_ns, int code) {
     const uint64_t t0 = globaltimer_ns();
-    // the clock is read every 64 polls; under a bound shorter than 1 ms at every poll
-    const uint32_t every = limit_ns < 1000000ull ? 0u : 63u;
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait_hint(bar, parity, 1000u)) return true;
-        if ((it & every) == 0) {
+        if ((it & 63u) == 0) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
                 *abort = 1;
