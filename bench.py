@@ -62,6 +62,9 @@ def parse_args(argv=None):
     ap.add_argument("--path", choices=["ws", "plain"], default="ws",
                     help="ws: gdn_forward_ws (shared prep through a workspace ring); "
                          "plain: gdn_forward (no workspace)")
+    ap.add_argument("--direction", choices=["causal", "bidir"], default="causal",
+                    help="causal: the forward scan; bidir: gdn_forward_bidir (forward plus backward "
+                         "scan from zero states, the dense checkpoint's form)")
     return ap.parse_args(argv)
 
 
@@ -239,13 +242,16 @@ def oracle_sample_size(inp, seconds, threads):
     return frames * fl
 
 
-def time_oracle(inp, n_tok, threads, repeats=1):
+def time_oracle(inp, n_tok, threads, repeats=1, bidir=False):
     from oracle import gdn_reference as R
     sub = slice_tokens(inp, n_tok)
     times = []
     for _ in range(repeats):
         t0 = time.perf_counter()
-        R.c_forward(sub, None, n_threads=threads, want_state=True)
+        if bidir:
+            R.c_bidirectional(sub, n_threads=threads)
+        else:
+            R.c_forward(sub, None, n_threads=threads, want_state=True)
         times.append(time.perf_counter() - t0)
     return times
 
@@ -254,12 +260,13 @@ def oracle_threads(w):
     return max(1, min(os.cpu_count() or 1, w.B * w.H))
 
 
-def cpu_baseline(w, inp, seconds):
+def cpu_baseline(w, inp, seconds, bidir=False):
     threads = oracle_threads(w)
-    n_tok = oracle_sample_size(inp, seconds, threads)
-    (dt,) = time_oracle(inp, n_tok, threads)
+    n_tok = oracle_sample_size(inp, seconds / (2 if bidir else 1), threads)
+    (dt,) = time_oracle(inp, n_tok, threads, bidir=bidir)
+    form = "forward plus backward token recurrence" if bidir else "token recurrence"
     return {"value": w.B * n_tok / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"float64 C token recurrence, first {n_tok} tokens of all {w.B * w.H} "
+            "sample": f"float64 C {form}, first {n_tok} tokens of all {w.B * w.H} "
                       f"(batch, head) chains of one layer, {threads} OpenMP threads "
                       f"(host has {os.cpu_count()} cores), {dt:.2f} s"}
 
@@ -331,13 +338,25 @@ def run_ours(args, w, rank, world, local):
     dims = (w.B, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.chunk_len)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), b.data_ptr(), None,
             st_out.data_ptr(), out.data_ptr())
+    bidir = args.direction == "bidir"
+    if bidir and (args.gate_mode == "frame" or args.path == "plain"):
+        raise SystemExit("--direction bidir takes the gate at every token and its own workspace")
     use_ws = args.path == "ws" and G.gdn_workspace_bytes(*dims[:5], w.chunk_len) > 0
-    ws = G.workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.chunk_len, device) if use_ws else None
-    ws_args = (ws.data_ptr(), ws.numel()) if use_ws else (None, 0)
+    if bidir:
+        ws = G.bidir_workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.chunk_len, device)
+    else:
+        ws = G.workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.chunk_len, device) if use_ws else None
+    ws_args = (ws.data_ptr(), ws.numel()) if ws is not None else (None, 0)
 
     gate_mode = 1 if args.gate_mode == "frame" else 0
 
     def layer_call():
+        if bidir:
+            st = lib.gdn_forward_bidir(q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), b.data_ptr(),
+                                       out.data_ptr(), *dims, *ws_args, sptr)
+            if st != 0:
+                raise G.GdnError(st, "gdn_forward_bidir")
+            return
         if gate_mode:
             st = lib.gdn_forward_gated(*ptrs, *dims, gate_mode, *ws_args, sptr)
         elif use_ws:
@@ -388,11 +407,13 @@ def run_ours(args, w, rank, world, local):
     avg_launch_s = statistics.mean(launch_ms) / 1e3
 
     peaks, peak_kind = measured_peaks()
-    abytes = algorithmic_bytes(w, state_in=False, state_out=True)
+    abytes = algorithmic_bytes(w, state_in=False, state_out=not bidir)
     achieved = abytes / avg_launch_s / 1e9
     traffic, traffic_kernel = recorded_traffic()
     path = G.gdn_bf16_path(w.d_k, w.d_v, w.chunk_len)
-    if use_ws:
+    if bidir:
+        kernel = "gdn_forward_bidir (one layer call: reverse copy, 2 x gdn_ring_kernel, combine)"
+    elif use_ws:
         kernel = "gdn_ring_kernel"
     else:
         kernel = "gdn_chunk_tc_kernel" if path == 1 else "chunk_ffma_kernel<bf16,64>"
@@ -409,29 +430,39 @@ def run_ours(args, w, rank, world, local):
                                            CHUNKED_FLOPS_PER_TOKEN_HEAD * w.B * w.T * w.H
                                            / (peaks["bf16_tflops"] * 1e12)) / avg_launch_s, 4)}
 
+    flops_scans = 2 if bidir else 1
+    roofline["tensor_flops_frac"] = round(roofline["tensor_flops_frac"] * flops_scans, 4)
+    roofline["roofline_frac"] = round(max(abytes / (peaks["hbm_gbs"] * 1e9),
+                                          flops_scans * CHUNKED_FLOPS_PER_TOKEN_HEAD * w.B * w.T * w.H
+                                          / (peaks["bf16_tflops"] * 1e12)) / avg_launch_s, 4)
+
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not bidir:
         e2e = run_e2e(lib, G, w, device, stream, (h_q, h_k, h_v, h_g, h_b),
                       (q, k, v, g, b), out, st_out, world, max(2, min(args.steps, 3)), ws)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, inp, args.cpu_seconds)
+        cpu = cpu_baseline(w, inp, args.cpu_seconds, bidir=bidir)
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": dict(workload_config(w, layers),
+                           direction=("forward plus backward scan (gdn_forward_bidir)" if bidir
+                                      else "forward scan"),
                            gate_placement=("once per frame, at its first token (gate_mode 1)" if gate_mode
                                            else "at every token of the frame"),
-                           api=(("gdn_forward_gated" if gate_mode else "gdn_forward_ws") +
-                                " (C ABI, device buffers, workspace "
-                                f"{ws.numel() / 2**20:.1f} MiB reused by every layer)") if use_ws
+                           api=("gdn_forward_bidir (C ABI, device buffers, workspace "
+                                f"{ws.numel() / 2**20:.1f} MiB reused by every layer)") if bidir
+                           else (("gdn_forward_gated" if gate_mode else "gdn_forward_ws") +
+                                 " (C ABI, device buffers, workspace "
+                                 f"{ws.numel() / 2**20:.1f} MiB reused by every layer)") if use_ws
                            else ("gdn_forward_gated" if gate_mode else "gdn_forward") +
                            " (C ABI, device buffers)"),
             "roofline": roofline,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * layers,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * layers * (4 if bidir else 1),
             "clocks": clock_rec}
     if world > 1:
         import torch.distributed as dist

@@ -125,6 +125,57 @@ int run_bf16_ws(const gdn::FwdParams& p, int chunk_len, void* ws, size_t ws_byte
     return to_status(gdn::launch_ring(p, ws, ws_bytes, stream));
 }
 
+// Layout of the bidirectional workspace (elem: 2 for bf16 I/O, 4 for fp32 I/O).
+int bidir_need(int B, int H, int T, int dk, int dv, int chunk_len, size_t elem, gdn::BidirLayout* L)
+{
+    size_t ring = 0;
+    if (elem == 2 && uses_ring(T, dk, dv, chunk_len)) {
+        const int st = workspace_need(B, H, dv, &ring);
+        if (st != GDN_OK) return st;
+    }
+    *L = gdn::bidir_layout(B, H, T, dk, dv, elem, ring);
+    return GDN_OK;
+}
+
+// Forward scan of the caller's inputs into out; backward scan as the forward kernel
+// over token-reversed copies in the workspace; then out += mirrored backward output.
+int run_bidir(const gdn::FwdParams& p, int chunk_len, size_t elem, void* ws, size_t ws_bytes,
+              cudaStream_t stream)
+{
+    if (p.T == 0) return GDN_OK;
+    if ((int64_t)p.H * (p.dk > p.dv ? p.dk : p.dv) * (int64_t)elem / 16 > INT32_MAX ||
+        (int64_t)p.B * p.T > 4 * (int64_t)INT32_MAX)
+        return GDN_ERR_UNSUPPORTED;
+    gdn::BidirLayout L;
+    int st = bidir_need(p.B, p.H, p.T, p.dk, p.dv, chunk_len, elem, &L);
+    if (st != GDN_OK) return st;
+    if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return GDN_ERR_INVALID_ARG;
+    const size_t nq = (size_t)p.B * p.T * p.H * p.dk * elem;
+    const size_t nv = (size_t)p.B * p.T * p.H * p.dv * elem;
+    const size_t ng = (size_t)p.B * p.F * p.H * sizeof(float);
+    const size_t nb = (size_t)p.B * p.T * p.H * sizeof(float);
+    if (overlaps(ws, L.total, p.q, nq) || overlaps(ws, L.total, p.k, nq) || overlaps(ws, L.total, p.v, nv) ||
+        overlaps(ws, L.total, p.gate, ng) || overlaps(ws, L.total, p.beta, nb) ||
+        overlaps(ws, L.total, p.out, nv))
+        return GDN_ERR_INVALID_ARG;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    if (gdn::launch_reverse_inputs(p, elem, w, L, stream) != cudaSuccess) return GDN_ERR_CUDA;
+    const gdn::FwdParams r = gdn::reversed_params(p, w, L);
+    const size_t ring_bytes = L.total - L.ring;
+    if (elem == 2) {
+        st = ring_bytes ? run_bf16_ws(p, chunk_len, w + L.ring, ring_bytes, stream) : run_bf16(p, chunk_len, stream);
+        if (st == GDN_OK)
+            st = ring_bytes ? run_bf16_ws(r, chunk_len, w + L.ring, ring_bytes, stream)
+                            : run_bf16(r, chunk_len, stream);
+        if (st != GDN_OK) return st;
+        return to_status(gdn::launch_combine<__nv_bfloat16>(p, w, L, stream));
+    }
+    st = to_status(gdn::launch_ffma<float>(p, chunk_len, stream));
+    if (st == GDN_OK) st = to_status(gdn::launch_ffma<float>(r, chunk_len, stream));
+    if (st != GDN_OK) return st;
+    return to_status(gdn::launch_combine<float>(p, w, L, stream));
+}
+
 int forward_host(const void* h_q, const void* h_k, const void* h_v,
                      const float* h_gate_logit, const float* h_beta_logit,
                      const float* h_state_in, float* h_state_out, void* h_out,
@@ -341,6 +392,46 @@ int gdn_state_step_ws(const void* q, const void* k, const void* v,
                       B, H, T, d_k, d_v, frame_len, chunk_len, &p);
     if (st != GDN_OK) return st;
     return run_bf16_ws(p, chunk_len, workspace, workspace_bytes, stream);
+}
+
+int gdn_bidir_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk_len, int elem_bytes,
+                              size_t* bytes)
+{
+    if (!bytes) return GDN_ERR_INVALID_ARG;
+    *bytes = 0;
+    if (elem_bytes != 2 && elem_bytes != 4) return GDN_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || T < 0 || (int64_t)B * H > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (!supported_dim(d_k) || !supported_dim(d_v)) return GDN_ERR_UNSUPPORTED;
+    if (chunk_len != 16 && chunk_len != 32 && chunk_len != 64) return GDN_ERR_UNSUPPORTED;
+    if (T == 0) return GDN_OK;
+    gdn::BidirLayout L;
+    const int st = bidir_need(B, H, T, d_k, d_v, chunk_len, (size_t)elem_bytes, &L);
+    if (st == GDN_OK) *bytes = L.total;
+    return st;
+}
+
+int gdn_forward_bidir(const void* q, const void* k, const void* v,
+                      const float* gate_logit, const float* beta_logit, void* out,
+                      int B, int H, int T, int d_k, int d_v, int frame_len, int chunk_len,
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    gdn::FwdParams p;
+    int st = validate(q, k, v, gate_logit, beta_logit, nullptr, nullptr, out, true, 2,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
+    if (st != GDN_OK) return st;
+    return run_bidir(p, chunk_len, 2, workspace, workspace_bytes, stream);
+}
+
+int gdn_forward_bidir_f32(const float* q, const float* k, const float* v,
+                          const float* gate_logit, const float* beta_logit, float* out,
+                          int B, int H, int T, int d_k, int d_v, int frame_len, int chunk_len,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    gdn::FwdParams p;
+    int st = validate(q, k, v, gate_logit, beta_logit, nullptr, nullptr, out, true, 4,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
+    if (st != GDN_OK) return st;
+    return run_bidir(p, chunk_len, 4, workspace, workspace_bytes, stream);
 }
 
 const char* gdn_status_string(int status)

@@ -3,4 +3,5 @@
 #include "gdn_ffma.cu"
 #include "gdn_tc.cu"
 #include "gdn_ring.cu"
+#include "gdn_bidir.cu"
 #include "gdn_api.cu"

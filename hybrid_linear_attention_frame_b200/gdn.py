@@ -22,8 +22,9 @@ GDN_ERR_TIMEOUT = -4
 EXPORTS = ("gdn_forward", "gdn_state_step", "gdn_forward_f32", "gdn_state_step_f32",
            "gdn_forward_host", "gdn_workspace_bytes", "gdn_forward_ws", "gdn_state_step_ws",
            "gdn_forward_host_ws", "gdn_forward_static_ws", "gdn_forward_gated",
-           "gdn_forward_gated_f32", "gdn_set_wait_limit_ns", "gdn_status_string", "gdn_get_last_device_status",
-           "gdn_bf16_path", "gdn_version")
+           "gdn_forward_gated_f32", "gdn_bidir_workspace_bytes", "gdn_forward_bidir",
+           "gdn_forward_bidir_f32", "gdn_set_wait_limit_ns", "gdn_status_string",
+           "gdn_get_last_device_status", "gdn_bf16_path", "gdn_version")
 
 
 class GdnError(RuntimeError):
@@ -76,6 +77,12 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.gdn_forward_gated.restype = I
     lib.gdn_forward_gated_f32.argtypes = [P] * 8 + [I] * 8 + [P]
     lib.gdn_forward_gated_f32.restype = I
+    lib.gdn_bidir_workspace_bytes.argtypes = [I] * 7 + [ctypes.POINTER(Z)]
+    lib.gdn_bidir_workspace_bytes.restype = I
+    lib.gdn_forward_bidir.argtypes = [P] * 6 + [I] * 7 + [P, Z, P]
+    lib.gdn_forward_bidir.restype = I
+    lib.gdn_forward_bidir_f32.argtypes = [P] * 6 + [I] * 7 + [P, Z, P]
+    lib.gdn_forward_bidir_f32.restype = I
     lib.gdn_status_string.argtypes = [I]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
@@ -241,6 +248,31 @@ def gdn_forward_gated_f32(q, k, v, gate_logit, beta_logit, state_in, state_out, 
     return _check(st, "gdn_forward_gated_f32", check)
 
 
+def gdn_bidir_workspace_bytes(B, H, T, d_k, d_v, chunk_len, elem_bytes=2) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().gdn_bidir_workspace_bytes(B, H, T, d_k, d_v, chunk_len, elem_bytes, ctypes.byref(n))
+    _check(st, "gdn_bidir_workspace_bytes", True)
+    return int(n.value)
+
+
+def gdn_forward_bidir(q, k, v, gate_logit, beta_logit, out, B, H, T, d_k, d_v, frame_len, chunk_len,
+                      workspace, workspace_bytes=None, stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().gdn_forward_bidir(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logit), _ptr(beta_logit), _ptr(out),
+                                  B, H, T, d_k, d_v, frame_len, chunk_len, _ptr(workspace), wb,
+                                  _stream(stream))
+    return _check(st, "gdn_forward_bidir", check)
+
+
+def gdn_forward_bidir_f32(q, k, v, gate_logit, beta_logit, out, B, H, T, d_k, d_v, frame_len, chunk_len,
+                          workspace, workspace_bytes=None, stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().gdn_forward_bidir_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logit), _ptr(beta_logit),
+                                      _ptr(out), B, H, T, d_k, d_v, frame_len, chunk_len, _ptr(workspace),
+                                      wb, _stream(stream))
+    return _check(st, "gdn_forward_bidir_f32", check)
+
+
 def gdn_set_wait_limit_ns(ns: int) -> int:
     return load().gdn_set_wait_limit_ns(int(ns))
 
@@ -268,6 +300,30 @@ def workspace(B, H, T, d_k, d_v, chunk_len=64, device="cuda"):
     if n == 0:
         return None
     return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def bidir_workspace(B, H, T, d_k, d_v, chunk_len=64, device="cuda", elem_bytes=2):
+    """A workspace tensor for gdn_forward_bidir(_f32) (None when T = 0)."""
+    import torch
+    n = gdn_bidir_workspace_bytes(B, H, T, d_k, d_v, chunk_len, elem_bytes)
+    if n == 0:
+        return None
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def forward_bidirectional(q, k, v, gate_logit, beta_logit, frame_len=880, chunk_len=64, stream=None, ws=None):
+    """out = forward scan + backward scan (zero states) for bf16 or float32 q/k/v;
+    ``ws`` from bidir_workspace, allocated here when not given."""
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    f32 = q.dtype == torch.float32
+    if ws is None:
+        ws = bidir_workspace(B, H, T, dk, dv, chunk_len, q.device, 4 if f32 else 2)
+    out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    fn = gdn_forward_bidir_f32 if f32 else gdn_forward_bidir
+    fn(q, k, v, gate_logit, beta_logit, out, B, H, T, dk, dv, frame_len, chunk_len, ws, stream=stream)
+    return out
 
 
 def forward(q, k, v, gate_logit, beta_logit, state_in=None, frame_len=880, chunk_len=64,

@@ -217,6 +217,48 @@ int gdn_forward_gated_f32(const float* q, const float* k, const float* v,
                           int B, int H, int T, int d_k, int d_v, int frame_len, int chunk_len,
                           int gate_mode, cudaStream_t stream);
 
+/*
+ * Bidirectional GDN for the dense (whole-clip) checkpoint.  The pages name a
+ * "bidirectional" checkpoint with full bidirectional attention over the clip
+ * (sglang cookbook SANA-WM page, dense-bidirectional section) but do not give the
+ * form; the library reads it as
+ *     o_t = S_t^T q_t + R_t^T q_t,
+ * S the forward scan of gdn_forward from a zero state, and R the same rule run from
+ * the last token to the first from a zero state,
+ *     R_t = a_t (I - beta_t k_t k_t^T) R_{t+1} + beta_t k_t v_t^T,  R_T = 0,
+ * every token keeping its own q, k, v, beta and its own frame's gate (applied at
+ * every token of the frame).  No state goes in or out.
+ *
+ * Layouts as gdn_forward (no state arguments).  The workspace (device, 256-byte
+ * aligned, not overlapping any argument, contents need no initialisation, owned by
+ * the caller and busy until the call's work on `stream` completes) holds the
+ * token-reversed copies of q, k, v, beta and the per-token gate logits, the backward
+ * scan's output and, for the bf16 entry, the ring of gdn_forward_ws where those sizes
+ * take it: gdn_bidir_workspace_bytes gives its size (about 1.5x the bytes of q, k
+ * and v; 0 when T = 0).  elem_bytes is 2 for gdn_forward_bidir, 4 for
+ * gdn_forward_bidir_f32.
+ *
+ * Work on `stream`: one copy kernel, the forward kernel twice (gdn_forward_ws's
+ * ring kernel where it applies, else gdn_forward's; the float32 kernel of
+ * gdn_forward_f32 for the _f32 entry), one combine kernel.  Rounding (bf16 entry):
+ * each scan's output is rounded to bf16, their sum is formed in fp32 and rounded to
+ * bf16 again.  Errors: as gdn_forward; a missing, misaligned, small or overlapping
+ * workspace gives GDN_ERR_INVALID_ARG; B*T above 4 * INT32_MAX gives
+ * GDN_ERR_UNSUPPORTED.  Nothing is enqueued on an error.
+ */
+int gdn_bidir_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk_len, int elem_bytes,
+                              size_t* bytes);
+
+int gdn_forward_bidir(const void* q, const void* k, const void* v,
+                      const float* gate_logit, const float* beta_logit, void* out,
+                      int B, int H, int T, int d_k, int d_v, int frame_len, int chunk_len,
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+int gdn_forward_bidir_f32(const float* q, const float* k, const float* v,
+                          const float* gate_logit, const float* beta_logit, float* out,
+                          int B, int H, int T, int d_k, int d_v, int frame_len, int chunk_len,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Human-readable text of a gdn_status value (static storage). */
 const char* gdn_status_string(int status);
 

@@ -5,6 +5,7 @@ Fake device addresses are used only for calls that must fail validation; no
 call here reaches a kernel launch.
 """
 
+import ctypes
 import os
 import re
 
@@ -177,3 +178,27 @@ def test_wait_limit_setter_needs_no_device():
     # sets a process-wide host value read at the next launch; 0 restores the default
     assert G.gdn_set_wait_limit_ns(1000) == G.GDN_OK
     assert G.gdn_set_wait_limit_ns(0) == G.GDN_OK
+
+
+def test_bidirectional_entry_points_validate_before_any_device_work():
+    lib = G.load()
+    n = ctypes.c_size_t(7)
+    assert lib.gdn_bidir_workspace_bytes(1, 2, 10, 64, 64, 64, 3, ctypes.byref(n)) == G.GDN_ERR_INVALID_ARG
+    assert n.value == 0
+    assert lib.gdn_bidir_workspace_bytes(1, 2, 10, 40, 64, 64, 2, ctypes.byref(n)) == G.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_bidir_workspace_bytes(1, 2, 0, 112, 112, 64, 2, ctypes.byref(n)) == G.GDN_OK
+    assert n.value == 0
+    # sizes without the ring need no device query: reversed q, k, v, gates, beta, backward output
+    assert G.gdn_bidir_workspace_bytes(1, 2, 10, 64, 64, 64) == 3 * 2560 + 2 * 256 + 2560
+    assert G.gdn_bidir_workspace_bytes(1, 2, 10, 64, 64, 64, 4) == 3 * 5120 + 2 * 256 + 5120
+    # null input, no workspace, bad chunk: refused before any CUDA call
+    st = lib.gdn_forward_bidir(None, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 1, 2, 10, 64, 64, 4, 64, 7 * A, 1 << 20, None)
+    assert st == G.GDN_ERR_INVALID_ARG
+    st = lib.gdn_forward_bidir(A, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 1, 2, 10, 64, 64, 4, 64, None, 0, None)
+    assert st == G.GDN_ERR_INVALID_ARG
+    st = lib.gdn_forward_bidir_f32(A, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 1, 2, 10, 64, 64, 4, 48, 7 * A, 1 << 20,
+                                   None)
+    assert st == G.GDN_ERR_UNSUPPORTED
+    # T = 0: nothing to do, nothing enqueued
+    st = lib.gdn_forward_bidir(A, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 1, 2, 0, 112, 112, 880, 64, None, 0, None)
+    assert st == G.GDN_OK

@@ -1,0 +1,153 @@
+"""GPU parity of the bidirectional entries (gdn_forward_bidir, gdn_forward_bidir_f32)
+against the float64 oracle's bidirectional form (forward scan plus backward scan
+from zero states, each token with its own frame's gate).  Bars: bf16 max-abs <= 2e-2
+and relative L2 <= 5e-3; float32 mode relative L2 <= 1e-4.
+
+Cases: sizes that take the ring kernel (d 112, ragged T, frames that do not divide
+T), the bf16 FFMA path (d 64 and 32, chunk 16/32/64), the float32 mode, single-token
+and sub-chunk sequences, more chains than CTA groups, the clip241 and minute-scale
+layers, and T = 0 (nothing is written).  Outputs are NaN-filled with guard bands,
+the workspace is filled with garbage first.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import gdn_reference as R
+from workloads import CLIP241, MINUTE, draw, make_inputs
+
+from gpu_util import assert_bf16_parity, assert_f32_parity, host, upload
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle(inp):
+    Bn, T, H, _ = inp.q.shape
+    if Bn * T * H <= 4000:
+        return R.bidirectional(inp)
+    return R.c_bidirectional(inp)
+
+
+def run_bidir(inp, device, chunk_len=64):
+    import torch
+    import hybrid_linear_attention_frame_b200 as G
+    q, k, v, g, b = upload(inp, device)
+    Bn, T, H, dk = inp.q.shape
+    dv = inp.v.shape[3]
+    f32 = inp.io_dtype == "f32"
+    guard = 64
+    n_out = Bn * T * H * dv
+    buf = torch.full((n_out + 2 * guard,), float("nan"), dtype=q.dtype, device=device)
+    buf[:guard] = 7.0
+    buf[-guard:] = 7.0
+    out = buf[guard:guard + n_out]
+    ws = G.bidir_workspace(Bn, H, T, dk, dv, chunk_len, device, 4 if f32 else 2)
+    if ws is not None:
+        ws.fill_(0xA5)
+    fn = G.gdn_forward_bidir_f32 if f32 else G.gdn_forward_bidir
+    fn(q, k, v, g, b, out, Bn, H, T, dk, dv, inp.frame_len, chunk_len, ws)
+    torch.cuda.synchronize()
+    assert G.gdn_get_last_device_status() == G.GDN_OK
+    assert torch.all(buf[:guard] == 7.0) and torch.all(buf[-guard:] == 7.0), "guard band overwritten"
+    o = host(out).reshape(Bn, T, H, dv)
+    assert not np.isnan(o).any(), "output not fully written"
+    return o
+
+
+def check_bf16(inp, device, what, chunk_len=64):
+    o = run_bidir(inp, device, chunk_len)
+    return assert_bf16_parity(o, oracle(inp), what)
+
+
+RNG_SEED = 31
+
+
+def cases_bf16():
+    rng = np.random.Generator(np.random.PCG64(RNG_SEED))
+    return {
+        "ring d112 ragged frames": (draw(rng, 2, 20, 700, 112, 112, 90, "bf16", 2.0, 0.5), 64),
+        "ring d112 strong decay": (draw(rng, 1, 4, 333, 112, 112, 50, "bf16", 0.0, 1.5), 64),
+        "ring d96 x 128": (draw(rng, 1, 6, 257, 96, 128, 64, "bf16", 1.0, 1.0), 64),
+        "ffma d64": (draw(rng, 1, 3, 200, 64, 64, 50, "bf16", 0.0, 1.0), 64),
+        "ffma d32 chunk 16": (draw(rng, 2, 2, 77, 32, 32, 7, "bf16", 0.5, 1.0), 16),
+        "ffma d48 x 64 chunk 32": (draw(rng, 1, 2, 95, 48, 64, 10, "bf16", 0.5, 1.0), 32),
+        "single token": (draw(rng, 1, 20, 1, 112, 112, 880, "bf16", 2.0, 0.5), 64),
+        "sub-chunk": (draw(rng, 1, 20, 37, 112, 112, 880, "bf16", 2.0, 0.5), 64),
+        "more chains than groups": (draw(rng, 4, 20, 130, 112, 112, 64, "bf16", 2.0, 0.5), 64),
+    }
+
+
+@pytest.mark.parametrize("name", sorted(cases_bf16()))
+def test_bidir_bf16_parity(cuda, name):
+    inp, chunk = cases_bf16()[name]
+    check_bf16(inp, cuda, f"bidir {name}", chunk)
+
+
+@pytest.mark.parametrize("dims", [(1, 3, 150, 112, 112, 40, 64), (2, 2, 70, 64, 32, 9, 32),
+                                  (1, 2, 1, 16, 16, 1, 16)])
+def test_bidir_f32_parity(cuda, dims):
+    Bn, H, T, dk, dv, fl, chunk = dims
+    rng = np.random.Generator(np.random.PCG64(RNG_SEED + T))
+    inp = draw(rng, Bn, H, T, dk, dv, fl, "f32", 0.5, 1.0)
+    o = run_bidir(inp, cuda, chunk)
+    assert_f32_parity(o, oracle(inp), f"bidir f32 {dims}")
+
+
+def test_bidir_is_forward_plus_reversed_forward_on_device(cuda):
+    """Library-level identity: the bidirectional output minus the library's own forward
+    output equals the library's forward output of the reversed sequence, mirrored
+    (float32 mode, frames of one token so that the reversal needs no regrouping)."""
+    import torch
+    import hybrid_linear_attention_frame_b200 as G
+    rng = np.random.Generator(np.random.PCG64(RNG_SEED + 1))
+    inp = draw(rng, 1, 3, 90, 64, 64, 1, "f32", 0.5, 1.0)
+    q, k, v, g, b = upload(inp, cuda)
+    o_bi = torch.from_numpy(run_bidir(inp, cuda)).to(cuda)
+    o_f, _ = G.forward(q, k, v, g, b, frame_len=1, want_state=False)
+    o_r, _ = G.forward(q.flip(1).contiguous(), k.flip(1).contiguous(), v.flip(1).contiguous(),
+                       g.flip(1).contiguous(), b.flip(1).contiguous(), frame_len=1, want_state=False)
+    torch.cuda.synchronize()
+    diff = (o_bi - o_f.double() - o_r.flip(1).double()).abs().max().item()
+    assert diff <= 1e-5 * max(1.0, o_bi.abs().max().item())
+
+
+def test_bidir_zero_tokens_writes_nothing(cuda):
+    import torch
+    import hybrid_linear_attention_frame_b200 as G
+    rng = np.random.Generator(np.random.PCG64(RNG_SEED + 3))
+    inp = draw(rng, 1, 2, 1, 112, 112, 880, "bf16", 2.0, 0.5)
+    q, k, v, g, b = upload(inp, cuda)          # real buffers, called with T = 0
+    sentinel = torch.full((16,), 3.0, dtype=torch.bfloat16, device=cuda)
+    assert G.gdn_bidir_workspace_bytes(1, 2, 0, 112, 112, 64) == 0
+    st = G.gdn_forward_bidir(q, k, v, g, b, sentinel, 1, 2, 0, 112, 112, 880, 64, None, 0)
+    torch.cuda.synchronize()
+    assert st == G.GDN_OK
+    assert torch.all(sentinel == 3.0)
+
+
+def test_bidir_workspace_checks(cuda):
+    import torch
+    import hybrid_linear_attention_frame_b200 as G
+    rng = np.random.Generator(np.random.PCG64(RNG_SEED + 2))
+    inp = draw(rng, 1, 4, 200, 112, 112, 50, "bf16", 2.0, 0.5)
+    q, k, v, g, b = upload(inp, cuda)
+    out = torch.empty_like(v)
+    need = G.gdn_bidir_workspace_bytes(1, 4, 200, 112, 112, 64)
+    ws = torch.empty(need + 512, dtype=torch.uint8, device=cuda)
+    args = (q, k, v, g, b, out, 1, 4, 200, 112, 112, 50, 64)
+    assert G.gdn_forward_bidir(*args, None, 0, check=False) == G.GDN_ERR_INVALID_ARG
+    assert G.gdn_forward_bidir(*args, ws, need - 1, check=False) == G.GDN_ERR_INVALID_ARG
+    assert G.gdn_forward_bidir(*args, ws[16:], need, check=False) == G.GDN_ERR_INVALID_ARG    # misaligned
+    assert G.gdn_forward_bidir(q, k, v, g, b, out, 1, 4, 200, 112, 112, 50, 64, out, need,
+                               check=False) == G.GDN_ERR_INVALID_ARG                        # overlaps out
+    assert G.gdn_forward_bidir(*args, ws, need, check=False) == G.GDN_OK
+    torch.cuda.synchronize()
+    assert G.gdn_get_last_device_status() == G.GDN_OK
+
+
+def test_bidir_clip241_full(cuda):
+    check_bf16(make_inputs(CLIP241), cuda, "bidir clip241")
+
+
+def test_bidir_minute_layer_full(cuda):
+    check_bf16(make_inputs(MINUTE), cuda, "bidir minute")

@@ -7,9 +7,10 @@ first wait that does not succeed at once gives up (nothing is broken: the
 producer is simply slower than the bound).  In the ring kernel the copy warp that
 waits, on a shared-memory counter, for the first record of its group polls the
 clock every ~1 us, while that record takes several microseconds of tensor-core work
-to appear, so the call times out every time.  In the fused kernel whether a wait
-outlasts 1 ns before its first clock check depends on scheduling, so either status
-is accepted there.  After each such call the default bound is restored and a
+to appear, so the call times out every time.  The fused kernel waits only on
+mbarriers with a suspend-time hint, and a hinted poll has been seen to return only
+once the phase completed, so its calls finish normally; either status is accepted
+there.  After each such call the default bound is restored and a
 normal call must match the untouched reference outputs bit for bit.
 """
 
