@@ -62,6 +62,9 @@ def parse_args(argv=None):
     ap.add_argument("--path", choices=["ws", "plain"], default="ws",
                     help="ws: gdn_forward_ws (shared prep through a workspace ring); "
                          "plain: gdn_forward (no workspace)")
+    ap.add_argument("--layer", choices=["gdn", "softmax"], default="gdn",
+                    help="gdn: the GDN layer; softmax: the chunk-causal softmax attention layer "
+                         "(gdn_softmax_attention, blocks of 3 frames, 2 cached blocks, 1 sink frame)")
     ap.add_argument("--direction", choices=["causal", "bidir"], default="causal",
                     help="causal: the forward scan; bidir: gdn_forward_bidir (forward plus backward "
                          "scan from zero states, the dense checkpoint's form)")
@@ -308,6 +311,142 @@ def workload_config(w, layers):
 
 
 # ----------------------------------------------------------------------------
+# softmax attention layer
+# ----------------------------------------------------------------------------
+
+ATTN_GEOMETRY = {"frames_per_block": 3, "cached_blocks": 2, "sink_frames": 1}
+
+
+def attention_flops(w) -> int:
+    """2 (d_k + d_v) flops per (query, visible key) pair: the QK^T and PV products.
+    A query of block b sees the sink frames and blocks max(0, b - cached) .. b."""
+    bl = ATTN_GEOMETRY["frames_per_block"] * w.frame_len
+    sink = min(w.T, ATTN_GEOMETRY["sink_frames"] * w.frame_len)
+    pairs = 0
+    for b in range(-(-w.T // bl)):
+        lo, hi = max(0, b - ATTN_GEOMETRY["cached_blocks"]) * bl, min(w.T, (b + 1) * bl)
+        keys = hi if lo <= sink else sink + hi - lo
+        pairs += (hi - b * bl) * keys
+    return 2 * (w.d_k + w.d_v) * pairs * w.B * w.H
+
+
+def attention_cpu_baseline(w, inp, seconds):
+    """The float64 oracle on one full query block of the layer (a bounded sample)."""
+    from oracle import attention_reference as A
+    bl = ATTN_GEOMETRY["frames_per_block"] * w.frame_len
+    b = min(-(-w.T // bl) - 1, 3)                   # a block with the full window (2 cached + sink)
+    t0 = time.perf_counter()
+    A.attention_block(inp.q[:, :, :1], inp.k[:, :, :1], inp.v[:, :, :1], b, w.frame_len,
+                      ATTN_GEOMETRY["frames_per_block"], ATTN_GEOMETRY["cached_blocks"],
+                      ATTN_GEOMETRY["sink_frames"])
+    per_head = max(time.perf_counter() - t0, 1e-3)
+    heads = max(1, min(w.H, int(seconds / per_head)))
+    t0 = time.perf_counter()
+    A.attention_block(inp.q[:, :, :heads], inp.k[:, :, :heads], inp.v[:, :, :heads], b, w.frame_len,
+                      ATTN_GEOMETRY["frames_per_block"], ATTN_GEOMETRY["cached_blocks"],
+                      ATTN_GEOMETRY["sink_frames"])
+    dt = time.perf_counter() - t0
+    nq = min(w.T, (b + 1) * bl) - b * bl
+    return {"value": w.B * nq * heads / w.H / dt, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"float64 numpy/BLAS softmax over the visible keys, query block {b} ({nq} queries) of "
+                      f"{heads} of {w.H} heads, scaled to the layer's heads, {dt:.2f} s"}
+
+
+def run_softmax(args, w, rank, world, local):
+    import numpy as np
+    import torch
+    import hybrid_linear_attention_frame_b200 as G
+    from workloads import bf16_bits, make_inputs
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init("nccl", world)
+    layers = args.layers or w.layers
+    lib = G.load()
+    inp = make_inputs(w)
+
+    def bf16(x):
+        return torch.from_numpy(bf16_bits(x).view(np.int16)).view(torch.bfloat16).to(device)
+    q, k, v = bf16(inp.q), bf16(inp.k), bf16(inp.v)
+    out = torch.empty_like(v)
+    stream = torch.cuda.current_stream(device)
+    sptr = stream.cuda_stream
+    geo = (w.frame_len, ATTN_GEOMETRY["frames_per_block"], ATTN_GEOMETRY["cached_blocks"],
+           ATTN_GEOMETRY["sink_frames"])
+
+    def layer_call():
+        st = lib.gdn_softmax_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), w.B, w.H, w.T,
+                                       w.d_k, w.d_v, *geo, sptr)
+        if st != 0:
+            raise G.GdnError(st, "gdn_softmax_attention")
+
+    for _ in range(args.warmup):
+        for _ in range(layers):
+            layer_call()
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps * layers)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        uuid = None
+    clocks = ClockSampler(uuid).start() if rank == 0 else None
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    t_start.record(stream)
+    i = 0
+    for _ in range(args.steps):
+        for _ in range(layers):
+            ev[i][0].record(stream)
+            layer_call()
+            ev[i][1].record(stream)
+            i += 1
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    clock_rec = clocks.stop() if clocks else None
+    dev_status = G.gdn_get_last_device_status()
+    if dev_status != G.GDN_OK:
+        raise G.GdnError(dev_status, "device status after the timed region")
+
+    elapsed_s = t_start.elapsed_time(t_end) / 1e3
+    value, slowest = aggregate_throughput(w.B * w.T * layers * args.steps, elapsed_s, world, device)
+    avg_launch_s = statistics.mean(s_.elapsed_time(e_) for (s_, e_) in ev) / 1e3
+    peaks, peak_kind = measured_peaks()
+    flops = attention_flops(w)
+    achieved = flops / avg_launch_s / 1e12
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None, "kernel": "chunk_attn_kernel",
+                "peak_source": f"{peak_kind} bf16_tflops_sustained (cuBLAS bf16 GEMM, seconds-long loop)",
+                "algorithmic_flops_per_launch": flops, "avg_launch_us": round(avg_launch_s * 1e6, 2),
+                "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4)}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = attention_cpu_baseline(w, inp, args.cpu_seconds)
+    cfg = workload_config(w, layers)
+    cfg["workload"] = (f"{w.name}: minute-scale SANA-WM softmax attention layer, B={w.B} H={w.H} T={w.T} "
+                       f"d_k=d_v={w.d_k}, blocks of 3 frames of {w.frame_len} tokens, 2 cached blocks, "
+                       f"1 sink frame, {layers} layers back-to-back per step")
+    cfg.update(ATTN_GEOMETRY)
+    cfg["api"] = "gdn_softmax_attention (C ABI, device buffers)"
+    for key in ("chunk_len", "gate_logits"):
+        cfg.pop(key, None)
+    line = {"metric": "softmax attention tokens/s per layer (20 heads x d112, chunk-causal with KV cache) "
+                      "on 1 B200; % of roofline",
+            "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(slowest * 1e3 / args.steps, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg, "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": None, "gpu_launches": args.steps * layers, "clocks": clock_rec}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+    return line if rank == 0 else None
+
+
+# ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
 
@@ -550,6 +689,8 @@ def main(argv=None):
         return run_profile_case(w, args.profile_tokens, args.path)
     if args.impl == "reference":
         line = run_reference(args, w, rank, world)
+    elif args.layer == "softmax":
+        line = run_softmax(args, w, rank, world, local)
     else:
         line = run_ours(args, w, rank, world, local)
     if line is not None:

@@ -434,6 +434,26 @@ int gdn_forward_bidir_f32(const float* q, const float* k, const float* v,
     return run_bidir(p, chunk_len, 4, workspace, workspace_bytes, stream);
 }
 
+int gdn_softmax_attention(const void* q, const void* k, const void* v, void* out,
+                          int B, int H, int T, int d_k, int d_v,
+                          int frame_len, int frames_per_block, int cached_blocks, int sink_frames,
+                          cudaStream_t stream)
+{
+    if (B < 1 || H < 1 || T < 0 || B > 65535 || H > 65535) return GDN_ERR_INVALID_ARG;
+    if (frame_len < 1 || frames_per_block < 1 || cached_blocks < 0 || sink_frames < 0) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)frame_len * frames_per_block > INT32_MAX / 2 || (int64_t)frame_len * sink_frames > INT32_MAX)
+        return GDN_ERR_INVALID_ARG;
+    if (!gdn::attn_supported(d_k, d_v)) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)T + 256 > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !out) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return GDN_ERR_INVALID_ARG;
+    const size_t nq = (size_t)B * T * H * d_k * 2, nv = (size_t)B * T * H * d_v * 2;
+    if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv)) return GDN_ERR_INVALID_ARG;
+    if (T == 0) return GDN_OK;
+    return to_status(gdn::launch_attn(q, k, v, out, B, H, T, d_k, d_v, frame_len * frames_per_block,
+                                      cached_blocks, frame_len * sink_frames, stream));
+}
+
 const char* gdn_status_string(int status)
 {
     switch (status) {

@@ -4,4 +4,5 @@
 #include "gdn_tc.cu"
 #include "gdn_ring.cu"
 #include "gdn_bidir.cu"
+#include "gdn_attn.cu"
 #include "gdn_api.cu"

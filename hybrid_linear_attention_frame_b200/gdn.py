@@ -23,7 +23,7 @@ EXPORTS = ("gdn_forward", "gdn_state_step", "gdn_forward_f32", "gdn_state_step_f
            "gdn_forward_host", "gdn_workspace_bytes", "gdn_forward_ws", "gdn_state_step_ws",
            "gdn_forward_host_ws", "gdn_forward_static_ws", "gdn_forward_gated",
            "gdn_forward_gated_f32", "gdn_bidir_workspace_bytes", "gdn_forward_bidir",
-           "gdn_forward_bidir_f32", "gdn_set_wait_limit_ns", "gdn_status_string",
+           "gdn_forward_bidir_f32", "gdn_softmax_attention", "gdn_set_wait_limit_ns", "gdn_status_string",
            "gdn_get_last_device_status", "gdn_bf16_path", "gdn_version")
 
 
@@ -83,6 +83,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.gdn_forward_bidir.restype = I
     lib.gdn_forward_bidir_f32.argtypes = [P] * 6 + [I] * 7 + [P, Z, P]
     lib.gdn_forward_bidir_f32.restype = I
+    lib.gdn_softmax_attention.argtypes = [P] * 4 + [I] * 9 + [P]
+    lib.gdn_softmax_attention.restype = I
     lib.gdn_status_string.argtypes = [I]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
@@ -273,6 +275,13 @@ def gdn_forward_bidir_f32(q, k, v, gate_logit, beta_logit, out, B, H, T, d_k, d_
     return _check(st, "gdn_forward_bidir_f32", check)
 
 
+def gdn_softmax_attention(q, k, v, out, B, H, T, d_k, d_v, frame_len, frames_per_block=3, cached_blocks=2,
+                          sink_frames=1, stream=None, check=True) -> int:
+    st = load().gdn_softmax_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, d_k, d_v, frame_len,
+                                      frames_per_block, cached_blocks, sink_frames, _stream(stream))
+    return _check(st, "gdn_softmax_attention", check)
+
+
 def gdn_set_wait_limit_ns(ns: int) -> int:
     return load().gdn_set_wait_limit_ns(int(ns))
 
@@ -323,6 +332,17 @@ def forward_bidirectional(q, k, v, gate_logit, beta_logit, frame_len=880, chunk_
     out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     fn = gdn_forward_bidir_f32 if f32 else gdn_forward_bidir
     fn(q, k, v, gate_logit, beta_logit, out, B, H, T, dk, dv, frame_len, chunk_len, ws, stream=stream)
+    return out
+
+
+def softmax_attention(q, k, v, frame_len=880, frames_per_block=3, cached_blocks=2, sink_frames=1, stream=None):
+    """out [B,T,H,d_v] = chunk-causal softmax attention of bf16 q, k [B,T,H,d_k], v [B,T,H,d_v]."""
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    gdn_softmax_attention(q, k, v, out, B, H, T, dk, dv, frame_len, frames_per_block, cached_blocks, sink_frames,
+                          stream)
     return out
 
 

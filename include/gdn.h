@@ -259,6 +259,30 @@ int gdn_forward_bidir_f32(const float* q, const float* k, const float* v,
                           int B, int H, int T, int d_k, int d_v, int frame_len, int chunk_len,
                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Chunk-causal softmax attention with a rolling KV cache: the softmax layers that
+ * SANA-WM interleaves with the GDN layers (sglang cookbook SANA-WM page, section 1
+ * architecture table, "softmax every 4 blocks"; pipeline-configuration table:
+ * num_frame_per_block 3, num_cached_blocks 2, sink_size 1 frame).  Per batch entry
+ * and head, over the whole sequence:
+ *     o_t = sum_{s in K(t)} softmax_s(q_t . k_s / sqrt(d_k)) v_s,
+ *     K(t) = [0, sink_frames * frame_len)
+ *            U [max(0, b - cached_blocks) * L, min(T, (b + 1) * L)),
+ * L = frames_per_block * frame_len, b = t / L: the sink frames, the cached blocks
+ * and the whole current block (causal across blocks, full inside one).  This is
+ * what streaming generation computes block by block with the cache.
+ *
+ * q, k: [B, T, H, d_k] bf16; v, out: [B, T, H, d_v] bf16; device pointers,
+ * 16-byte aligned; out must not overlap q, k or v.  d_k, d_v in 80..128, multiples
+ * of 16 (GDN_ERR_UNSUPPORTED otherwise); B, H <= 65535.  Scores and the softmax in
+ * fp32, P rounded to bf16 for the P V product, output rounded to bf16.  T = 0 does
+ * nothing.  One kernel launch on `stream`; no workspace.  Errors as gdn_forward.
+ */
+int gdn_softmax_attention(const void* q, const void* k, const void* v, void* out,
+                          int B, int H, int T, int d_k, int d_v,
+                          int frame_len, int frames_per_block, int cached_blocks, int sink_frames,
+                          cudaStream_t stream);
+
 /* Human-readable text of a gdn_status value (static storage). */
 const char* gdn_status_string(int status);
 

@@ -22,9 +22,9 @@ the cached blocks and the whole current block (keys after t inside the current
 block included: "chunk-causal" is causal across blocks, full within one).  The
 scale 1/sqrt(d_k) is the usual one; the pages print none.
 
-``chunk_causal_attention`` evaluates this block by block (all queries of a block
-share K); ``attention_one_query`` evaluates one query, for sampled checks of
-full-size outputs.
+``chunk_causal_attention`` evaluates this block by block (``attention_block``: all
+queries of a block share K); ``attention_one_query`` evaluates one query, for
+sampled checks of full-size outputs.
 """
 
 import math
@@ -49,22 +49,29 @@ def _softmax_rows(scores):
     return e / np.sum(e, axis=-1, keepdims=True)
 
 
-def chunk_causal_attention(q, k, v, frame_len, frames_per_block=3, cached_blocks=2, sink_frames=1,
-                           scale=None):
-    """q, k [B, T, H, d_k], v [B, T, H, d_v] -> out [B, T, H, d_v] (float64)."""
-    q = np.asarray(q, np.float64)
-    k = np.asarray(k, np.float64)
-    v = np.asarray(v, np.float64)
+def attention_block(q, k, v, b, frame_len, frames_per_block=3, cached_blocks=2, sink_frames=1, scale=None):
+    """Outputs of query block b alone: [B, len(block), H, d_v] (float64)."""
     B, T, H, dk = q.shape
     sc = 1.0 / math.sqrt(dk) if scale is None else scale
     bl = frames_per_block * frame_len
-    out = np.zeros(v.shape)
+    t0, t1 = b * bl, min(T, (b + 1) * bl)
+    keys = block_keys(b, T, frame_len, frames_per_block, cached_blocks, sink_frames)
+    qb = np.asarray(q[:, t0:t1], np.float64).transpose(0, 2, 1, 3)          # [B, H, t, d_k]
+    kb = np.asarray(k[:, keys], np.float64).transpose(0, 2, 3, 1)           # [B, H, d_k, s]
+    vb = np.asarray(v[:, keys], np.float64).transpose(0, 2, 1, 3)           # [B, H, s, d_v]
+    p = _softmax_rows((qb @ kb) * sc)                                       # [B, H, t, s]
+    return (p @ vb).transpose(0, 2, 1, 3)
+
+
+def chunk_causal_attention(q, k, v, frame_len, frames_per_block=3, cached_blocks=2, sink_frames=1,
+                           scale=None):
+    """q, k [B, T, H, d_k], v [B, T, H, d_v] -> out [B, T, H, d_v] (float64)."""
+    B, T, H, dk = np.shape(q)
+    bl = frames_per_block * frame_len
+    out = np.zeros(np.shape(v)[:3] + (np.shape(v)[3],))
     for b in range(-(-T // bl)):
-        t0, t1 = b * bl, min(T, (b + 1) * bl)
-        keys = block_keys(b, T, frame_len, frames_per_block, cached_blocks, sink_frames)
-        s = np.einsum("bthd,bshd->bhts", q[:, t0:t1], k[:, keys]) * sc
-        p = _softmax_rows(s)
-        out[:, t0:t1] = np.einsum("bhts,bshd->bthd", p, v[:, keys])
+        out[:, b * bl:min(T, (b + 1) * bl)] = attention_block(q, k, v, b, frame_len, frames_per_block,
+                                                              cached_blocks, sink_frames, scale)
     return out
 
 
