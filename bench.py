@@ -680,11 +680,35 @@ def run_profile_case(w, tokens, path="ws"):
     return 0 if status == G.GDN_OK else 1
 
 
+def run_profile_case_softmax(w, tokens):
+    """Two softmax-attention layer calls on the first `tokens` tokens (profiling case)."""
+    import numpy as np
+    import torch
+    import hybrid_linear_attention_frame_b200 as G
+    from workloads import bf16_bits, make_inputs
+    inp = make_inputs(w, T=tokens)
+
+    def bf16(x):
+        return torch.from_numpy(bf16_bits(x).view(np.int16).copy()).view(torch.bfloat16).cuda()
+    q, k, v = bf16(inp.q), bf16(inp.k), bf16(inp.v)
+    out = torch.empty_like(v)
+    for _ in range(2):
+        G.gdn_softmax_attention(q, k, v, out, w.B, w.H, tokens, w.d_k, w.d_v, w.frame_len,
+                                ATTN_GEOMETRY["frames_per_block"], ATTN_GEOMETRY["cached_blocks"],
+                                ATTN_GEOMETRY["sink_frames"])
+    torch.cuda.synchronize()
+    status = G.gdn_get_last_device_status()
+    print(f"softmax profile case: T={tokens}, device status {status}")
+    return 0 if status == G.GDN_OK else 1
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_env()
     from workloads import MINUTE
     w = MINUTE
+    if args.profile_tokens > 0 and args.layer == "softmax":
+        return run_profile_case_softmax(w, args.profile_tokens)
     if args.profile_tokens > 0:
         return run_profile_case(w, args.profile_tokens, args.path)
     if args.impl == "reference":
