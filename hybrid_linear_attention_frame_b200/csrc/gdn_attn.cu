@@ -247,31 +247,46 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
         for (int c = 0; c < kBN / 16; ++c)
             tmem_ld16(lane_base + kColS + 128u * (j & 1) + 16u * c, *reinterpret_cast<float(*)[16]>(&x[16 * c]));
+        // Is the whole tile inside this row's key set?  (Then no per-key mask.)
+        bool full;
+        if (sink_tile) full = s0 + kBN <= sink;
+        else if (split) full = s0 >= ws && s0 + kBN <= we;
+        else full = (ws <= sink) ? (s0 + kBN <= max(sink, we))
+                                 : (s0 + kBN <= sink || (s0 >= ws && s0 + kBN <= we));
         tmem_wait_ld();
-        float mt = -INFINITY;
+        if (!full) {
 #pragma unroll
-        for (int i = 0; i < kBN; ++i) {
-            const int s = s0 + i;
-            const bool valid = sink_tile ? (s < sink)
-                                         : (s < T && ((!split && s < sink) || (s >= ws && s < we)));
-            x[i] = valid ? x[i] * a.scale_log2 : -INFINITY;
-            mt = fmaxf(mt, x[i]);
+            for (int i = 0; i < kBN; ++i) {
+                const int s = s0 + i;
+                const bool valid = sink_tile ? (s < sink)
+                                             : (s < T && ((!split && s < sink) || (s >= ws && s < we)));
+                x[i] = valid ? x[i] : -INFINITY;
+            }
         }
+        // maximum of the raw scores in 4 independent chains (the scale is positive)
+        float mx[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx[e] = x[e];
+#pragma unroll
+        for (int i = 4; i < kBN; ++i) mx[i & 3] = fmaxf(mx[i & 3], x[i]);
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.scale_log2;
         const bool move = mt > m_ref + kMoveRef;
         float alpha = 1.0f;
         if (move) {
             alpha = ex2(m_ref - mt);
             m_ref = mt;
         }
-        const float mr = (m_ref == -INFINITY) ? 0.0f : m_ref;
-        float sum = 0.0f;
+        const float neg_mr = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+        float sm[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[kBN / 2];
 #pragma unroll
         for (int i = 0; i < kBN / 2; ++i) {
-            const float p0 = ex2(x[2 * i] - mr), p1 = ex2(x[2 * i + 1] - mr);
-            sum += p0 + p1;
+            const float p0 = ex2(fmaf(x[2 * i], a.scale_log2, neg_mr));
+            const float p1 = ex2(fmaf(x[2 * i + 1], a.scale_log2, neg_mr));
+            sm[i & 3] += p0 + p1;
             pk[i] = pack_bf16x2(p0, p1);
         }
+        const float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);
         l = l * alpha + sum;
         // ---- the previous P V must be done: P's buffer is reused and O may be rescaled ----
         if (j > 0) {
