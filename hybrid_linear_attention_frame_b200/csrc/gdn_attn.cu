@@ -9,8 +9,9 @@
 //
 // the sink frames, the cached blocks and the whole current block.
 //
-// One CTA of 128 threads per (128 queries, head, batch entry); thread r owns query
-// row r and TMEM lane r.  For each key tile of 128 tokens:
+// One CTA of 256 threads per (128 queries, head, batch entry); threads r and r + 128
+// share query row r (TMEM lane r), each taking 64 of a tile's keys and half of the
+// output columns.  For each key tile of 128 tokens:
 //   S = Q K^T on the tensor cores into TMEM (two buffers: the next tile's S runs
 //     while this tile's softmax does),
 //   the softmax in registers against a lazily moved reference maximum (it moves
@@ -29,7 +30,8 @@ namespace attn {
 
 using namespace sm100;
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;                  // two threads per query row
+constexpr int kHalfKeys = 64;                  // keys of a tile per thread
 constexpr int kBM = 128;                       // queries per CTA
 constexpr int kBN = 128;                       // keys per tile
 constexpr uint32_t kBox = 128u * 128u;         // one 64-column SW128 box of 128 rows: 16 KB
@@ -44,7 +46,8 @@ enum : uint32_t { kBarQ = 0, kBarK = 1, kBarV = kBarK + kKStages, kBarS = kBarV 
                   kNumBars = kBarPV + 1 };
 constexpr uint32_t kOffAbort = kOffBar + 8u * kNumBars;
 constexpr uint32_t kOffTmemSlot = kOffAbort + 8u;
-constexpr uint32_t kSmemBytes = kOffTmemSlot + 8u + 1024u;     // + slack for 1024-byte alignment
+constexpr uint32_t kOffX = kOffTmemSlot + 16u;                 // 256 floats: the two halves' exchange
+constexpr uint32_t kSmemBytes = kOffX + 4u * kThreads + 1024u; // + slack for 1024-byte alignment
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "SW128 tiles need 1024-B alignment");
 
@@ -52,7 +55,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;                  // two 128-column score buffers
 constexpr uint32_t kColO = 256;                // the d_v-column output accumulator
 constexpr float kMoveRef = 8.0f;               // log2 units: p stays below 2^8
-constexpr uint32_t kBarGroup = 1;              // named barrier of the 128 threads
+constexpr uint32_t kBarGroup = 1;              // named barrier of all the CTA's threads
 
 constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);
 
@@ -146,8 +149,9 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int n = nA + (w_hi - startB + kBN - 1) / kBN;
     auto tile_start = [&](int j) { return j < nA ? kBN * j : startB + kBN * (j - nA); };
 
-    // ---- this thread's query row and its own key set ----
-    const int t = t0 + tid;
+    // ---- this thread's query row, half of the keys and its row's key set ----
+    const int row = tid & (kBM - 1), half = tid / kBM;
+    const int t = t0 + row;
     const int te = min(t, T - 1);
     const int ws = max(0, te / bl - a.cached) * bl;
     const int we = min(T, (te / bl + 1) * bl);
@@ -168,7 +172,9 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gb + kOffTmemSlot);
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);   // warp w reads lanes 32 (w % 4) ..
+    float* xchg = reinterpret_cast<float*>(gb + kOffX);
+    const int nco = a.dv / 16, c_lo = half ? (nco + 1) / 2 : 0, c_hi = half ? nco : (nco + 1) / 2;
     const uint32_t idpv = idesc_bf16(128, a.dv, false, true);
     const int nks = a.dk / 16;
 
@@ -241,36 +247,39 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (!group_all(kBarGroup, kThreads, ok)) { alive = false; break; }
         s_waited = j + 1;
         tc_fence_after();
-        const int s0 = tile_start(j);
+        const int s0 = tile_start(j) + kHalfKeys * half;     // this thread's first key
         const bool sink_tile = j < nA;
-        float x[kBN];
+        float x[kHalfKeys];
 #pragma unroll
-        for (int c = 0; c < kBN / 16; ++c)
-            tmem_ld16(lane_base + kColS + 128u * (j & 1) + 16u * c, *reinterpret_cast<float(*)[16]>(&x[16 * c]));
-        // Is the whole tile inside this row's key set?  (Then no per-key mask.)
+        for (int c = 0; c < kHalfKeys / 16; ++c)
+            tmem_ld16(lane_base + kColS + 128u * (j & 1) + (uint32_t)(kHalfKeys * half) + 16u * c,
+                      *reinterpret_cast<float(*)[16]>(&x[16 * c]));
+        // Are all of this thread's keys inside its row's key set?  (Then no per-key mask.)
         bool full;
-        if (sink_tile) full = s0 + kBN <= sink;
-        else if (split) full = s0 >= ws && s0 + kBN <= we;
-        else full = (ws <= sink) ? (s0 + kBN <= max(sink, we))
-                                 : (s0 + kBN <= sink || (s0 >= ws && s0 + kBN <= we));
+        if (sink_tile) full = s0 + kHalfKeys <= sink;
+        else if (split) full = s0 >= ws && s0 + kHalfKeys <= we;
+        else full = (ws <= sink) ? (s0 + kHalfKeys <= max(sink, we))
+                                 : (s0 + kHalfKeys <= sink || (s0 >= ws && s0 + kHalfKeys <= we));
         tmem_wait_ld();
         if (!full) {
 #pragma unroll
-            for (int i = 0; i < kBN; ++i) {
+            for (int i = 0; i < kHalfKeys; ++i) {
                 const int s = s0 + i;
                 const bool valid = sink_tile ? (s < sink)
                                              : (s < T && ((!split && s < sink) || (s >= ws && s < we)));
                 x[i] = valid ? x[i] : -INFINITY;
             }
         }
-        // maximum of the raw scores in 4 independent chains (the scale is positive)
+        // maximum of the raw scores (the scale is positive) over both halves of the row
         float mx[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) mx[e] = x[e];
 #pragma unroll
-        for (int i = 4; i < kBN; ++i) mx[i & 3] = fmaxf(mx[i & 3], x[i]);
-        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.scale_log2;
-        const bool move = mt > m_ref + kMoveRef;
+        for (int i = 4; i < kHalfKeys; ++i) mx[i & 3] = fmaxf(mx[i & 3], x[i]);
+        xchg[tid] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        named_bar_sync(kBarGroup, kThreads);
+        const float mt = fmaxf(xchg[tid], xchg[tid ^ kBM]) * a.scale_log2;
+        const bool move = mt > m_ref + kMoveRef;   // the same decision in both threads of the row
         float alpha = 1.0f;
         if (move) {
             alpha = ex2(m_ref - mt);
@@ -278,15 +287,15 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         const float neg_mr = (m_ref == -INFINITY) ? 0.0f : -m_ref;
         float sm[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[kBN / 2];
+        uint32_t pk[kHalfKeys / 2];
 #pragma unroll
-        for (int i = 0; i < kBN / 2; ++i) {
+        for (int i = 0; i < kHalfKeys / 2; ++i) {
             const float p0 = ex2(fmaf(x[2 * i], a.scale_log2, neg_mr));
             const float p1 = ex2(fmaf(x[2 * i + 1], a.scale_log2, neg_mr));
             sm[i & 3] += p0 + p1;
             pk[i] = pack_bf16x2(p0, p1);
         }
-        const float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);
+        const float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);     // this half's part of the row sum
         l = l * alpha + sum;
         // ---- the previous P V must be done: P's buffer is reused and O may be rescaled ----
         if (j > 0) {
@@ -301,7 +310,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (__any_sync(0xffffffffu, move && j > 0)) {
             const float f = (move && j > 0) ? alpha : 1.0f;
 #pragma unroll 1
-            for (int c = 0; c < a.dv / 16; ++c) {
+            for (int c = c_lo; c < c_hi; ++c) {
                 float o[16];
                 tmem_ld16(lane_base + kColO + 16u * c, o);
                 tmem_wait_ld();
@@ -311,16 +320,13 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             tmem_wait_st();
         }
-        // ---- P row (128 keys, bf16) into the K-major SW128 operand ----
+        // ---- this thread's 64 keys of the P row (bf16) into its box of the K-major SW128 operand ----
         {
-            const uint32_t prow = base + kOffP + (uint32_t)tid * 128u;
+            const uint32_t prow = base + kOffP + (uint32_t)half * kBox + (uint32_t)row * 128u;
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    st_shared_v4(prow + (uint32_t)hh * kBox + ((uint32_t)(c ^ (tid & 7)) << 4),
-                                 pk[32 * hh + 4 * c], pk[32 * hh + 4 * c + 1], pk[32 * hh + 4 * c + 2],
-                                 pk[32 * hh + 4 * c + 3]);
+            for (int c = 0; c < 8; ++c)
+                st_shared_v4(prow + ((uint32_t)(c ^ (row & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                             pk[4 * c + 3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -345,11 +351,13 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (alive) {
             pv_waited = n;
             tc_fence_after();
-            const float inv = 1.0f / l;
+            xchg[tid] = l;                       // the row sum is the two halves' parts
+            named_bar_sync(kBarGroup, kThreads);
+            const float inv = 1.0f / (xchg[tid] + xchg[tid ^ kBM]);
             __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) +
                                   (((size_t)bb * T + (size_t)t) * a.H + h) * (size_t)a.dv;
 #pragma unroll 1
-            for (int c = 0; c < a.dv / 16; ++c) {
+            for (int c = c_lo; c < c_hi; ++c) {
                 float o[16];
                 tmem_ld16(lane_base + kColO + 16u * c, o);
                 tmem_wait_ld();
