@@ -202,3 +202,25 @@ def test_bidirectional_entry_points_validate_before_any_device_work():
     # T = 0: nothing to do, nothing enqueued
     st = lib.gdn_forward_bidir(A, 2 * A, 3 * A, 4 * A, 5 * A, 6 * A, 1, 2, 0, 112, 112, 880, 64, None, 0, None)
     assert st == G.GDN_OK
+
+
+def test_softmax_attention_validates_before_any_device_work():
+    lib = G.load()
+    args = (A, 2 * A, 3 * A, 5 * A)
+    # unsupported head sizes, bad geometry, null or misaligned pointers, overlapping output
+    assert lib.gdn_softmax_attention(*args, 1, 2, 64, 64, 64, 16, 3, 2, 1, None) == G.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_softmax_attention(*args, 1, 2, 64, 112, 72, 16, 3, 2, 1, None) == G.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_softmax_attention(*args, 1, 2, 64, 112, 112, 0, 3, 2, 1, None) == G.GDN_ERR_INVALID_ARG
+    assert lib.gdn_softmax_attention(*args, 1, 2, 64, 112, 112, 16, 0, 2, 1, None) == G.GDN_ERR_INVALID_ARG
+    assert lib.gdn_softmax_attention(*args, 1, 2, 64, 112, 112, 16, 3, -1, 1, None) == G.GDN_ERR_INVALID_ARG
+    assert lib.gdn_softmax_attention(*args, 1, 2, 64, 112, 112, 16, 3, 2, -1, None) == G.GDN_ERR_INVALID_ARG
+    assert lib.gdn_softmax_attention(*args, 0, 2, 64, 112, 112, 16, 3, 2, 1, None) == G.GDN_ERR_INVALID_ARG
+    assert lib.gdn_softmax_attention(*args, 1, 70000, 64, 112, 112, 16, 3, 2, 1, None) == G.GDN_ERR_INVALID_ARG
+    assert lib.gdn_softmax_attention(None, 2 * A, 3 * A, 5 * A, 1, 2, 64, 112, 112, 16, 3, 2, 1,
+                                     None) == G.GDN_ERR_INVALID_ARG
+    assert lib.gdn_softmax_attention(A + 8, 2 * A, 3 * A, 5 * A, 1, 2, 64, 112, 112, 16, 3, 2, 1,
+                                     None) == G.GDN_ERR_INVALID_ARG
+    assert lib.gdn_softmax_attention(A, 2 * A, 3 * A, A + 64, 1, 2, 64, 112, 112, 16, 3, 2, 1,
+                                     None) == G.GDN_ERR_INVALID_ARG
+    # T = 0: nothing to do, nothing enqueued
+    assert lib.gdn_softmax_attention(*args, 1, 2, 0, 112, 112, 16, 3, 2, 1, None) == G.GDN_OK

@@ -68,3 +68,23 @@ def test_two_rank_gloo_aggregate_takes_slowest_rank():
 def test_reference_arm_other_ranks_do_no_work():
     args = bench.parse_args(["--impl", "reference"])
     assert bench.run_reference(args, MINUTE, rank=1, world=2) is None
+
+
+def test_attention_flops_match_the_oracle_key_sets():
+    """The bench's closed-form count of visible (query, key) pairs against the oracle's
+    key sets, block by block, at the minute-scale shape and a ragged one."""
+    from oracle import attention_reference as A
+    from workloads import MINUTE
+    for w in (MINUTE, MINUTE.with_(T=5000, H=3)):
+        bl = 3 * w.frame_len
+        pairs = sum((min(w.T, (b + 1) * bl) - b * bl) * len(A.block_keys(b, w.T, w.frame_len, 3, 2, 1))
+                    for b in range(-(-w.T // bl)))
+        assert bench.attention_flops(w) == 2 * (w.d_k + w.d_v) * pairs * w.B * w.H
+    assert bench.attention_flops(MINUTE) == 8132067328000
+
+
+def test_softmax_and_bidir_modes_parse():
+    a = bench.parse_args(["--layer", "softmax", "--steps", "2"])
+    assert a.layer == "softmax" and a.direction == "causal"
+    a = bench.parse_args(["--direction", "bidir"])
+    assert a.layer == "gdn" and a.direction == "bidir"
