@@ -47,6 +47,14 @@
  * Every pointer to q, k, v, out and the state must be 16-byte aligned; the
  * logit pointers 4-byte aligned.  `out` must not overlap any input.
  * state_in == state_out is allowed (in-place update).
+ *
+ * Beyond the forward layer the library also provides, each documented at its
+ * declaration: the workspace and allocation-free variants of the forward pass
+ * (gdn_forward_ws, gdn_state_step_ws, gdn_forward_host_ws, gdn_forward_static_ws),
+ * the other gate placement (gdn_forward_gated*), the bidirectional form of the
+ * dense checkpoint (gdn_forward_bidir*), the chunk-causal softmax attention layer
+ * with its rolling KV cache (gdn_softmax_attention), and the status and wait-bound
+ * controls (gdn_get_last_device_status, gdn_set_wait_limit_ns).
  */
 #ifndef GDN_H
 #define GDN_H
