@@ -275,26 +275,42 @@ def cpu_baseline(w, inp, seconds, bidir=False):
 
 
 def run_reference(args, w, rank, world):
-    """Reference arm: the float64 CPU oracle on bounded samples of the same workload."""
+    """Reference arm: the float64 CPU oracle on bounded samples of the same workload
+    (the GDN layer, its bidirectional form, or the softmax layer, as the flags say)."""
     if rank != 0:
         return None
     from workloads import make_inputs
     inp = make_inputs(w)
     threads = oracle_threads(w)
     budget = 150.0 / max(1, args.steps + args.warmup)      # whole run within a few minutes
-    n_tok = oracle_sample_size(inp, min(args.cpu_seconds, budget), threads)
-    time_oracle(inp, n_tok, threads, repeats=args.warmup)
-    times = time_oracle(inp, n_tok, threads, repeats=args.steps)
-    per_step = sum(times) / len(times)
-    value = w.B * n_tok / per_step
-    sample = (f"float64 C token recurrence, first {n_tok} tokens of all {w.B * w.H} chains "
-              f"of one layer per step, {threads} OpenMP threads (host has {os.cpu_count()} cores)")
-    return {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
+    layers = args.layers or w.layers
+    if args.layer == "softmax":
+        per_call = min(args.cpu_seconds, budget)
+        for _ in range(args.warmup):
+            attention_cpu_baseline(w, inp, per_call)
+        runs = [attention_cpu_baseline(w, inp, per_call) for _ in range(args.steps)]
+        value = statistics.mean(r["value"] for r in runs)
+        per_step = w.B * w.T / value
+        sample = runs[-1]["sample"] + " per step"
+        metric, config, cores = ATTN_METRIC, attention_config(w, layers), os.cpu_count()
+    else:
+        bidir = args.direction == "bidir"
+        n_tok = oracle_sample_size(inp, min(args.cpu_seconds, budget) / (2 if bidir else 1), threads)
+        time_oracle(inp, n_tok, threads, repeats=args.warmup, bidir=bidir)
+        times = time_oracle(inp, n_tok, threads, repeats=args.steps, bidir=bidir)
+        per_step = sum(times) / len(times)
+        value = w.B * n_tok / per_step
+        form = "forward plus backward token recurrence" if bidir else "token recurrence"
+        sample = (f"float64 C {form}, first {n_tok} tokens of all {w.B * w.H} chains "
+                  f"of one layer per step, {threads} OpenMP threads (host has {os.cpu_count()} cores)")
+        metric, config, cores = METRIC, workload_config(w, layers), threads
+        if bidir:
+            config["direction"] = "forward plus backward scan (gdn_forward_bidir)"
+    return {"metric": metric, "value": value, "unit": UNIT, "impl": "reference",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w, args.layers or w.layers),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -328,6 +344,22 @@ def attention_flops(w) -> int:
         keys = hi if lo <= sink else sink + hi - lo
         pairs += (hi - b * bl) * keys
     return 2 * (w.d_k + w.d_v) * pairs * w.B * w.H
+
+
+ATTN_METRIC = ("softmax attention tokens/s per layer (20 heads x d112, chunk-causal with KV cache) "
+               "on 1 B200; % of roofline")
+
+
+def attention_config(w, layers):
+    cfg = workload_config(w, layers)
+    cfg["workload"] = (f"{w.name}: minute-scale SANA-WM softmax attention layer, B={w.B} H={w.H} T={w.T} "
+                       f"d_k=d_v={w.d_k}, blocks of 3 frames of {w.frame_len} tokens, 2 cached blocks, "
+                       f"1 sink frame, {layers} layers back-to-back per step")
+    cfg.update(ATTN_GEOMETRY)
+    cfg["api"] = "gdn_softmax_attention (C ABI, device buffers)"
+    for key in ("chunk_len", "gate_logits"):
+        cfg.pop(key, None)
+    return cfg
 
 
 def attention_cpu_baseline(w, inp, seconds):
@@ -425,16 +457,8 @@ def run_softmax(args, w, rank, world, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = attention_cpu_baseline(w, inp, args.cpu_seconds)
-    cfg = workload_config(w, layers)
-    cfg["workload"] = (f"{w.name}: minute-scale SANA-WM softmax attention layer, B={w.B} H={w.H} T={w.T} "
-                       f"d_k=d_v={w.d_k}, blocks of 3 frames of {w.frame_len} tokens, 2 cached blocks, "
-                       f"1 sink frame, {layers} layers back-to-back per step")
-    cfg.update(ATTN_GEOMETRY)
-    cfg["api"] = "gdn_softmax_attention (C ABI, device buffers)"
-    for key in ("chunk_len", "gate_logits"):
-        cfg.pop(key, None)
-    line = {"metric": "softmax attention tokens/s per layer (20 heads x d112, chunk-causal with KV cache) "
-                      "on 1 B200; % of roofline",
+    cfg = attention_config(w, layers)
+    line = {"metric": ATTN_METRIC,
             "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(slowest * 1e3 / args.steps, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg, "roofline": roofline,
