@@ -17,6 +17,8 @@ bool ring_supported(int dk, int dv, int chunk_len);
 cudaError_t ring_groups(int BH, int dv, int* groups);
 size_t ring_workspace_bytes(int G, int dv);
 cudaError_t launch_ring(const FwdParams& p, void* ws, size_t ws_bytes, cudaStream_t stream);
+bool seq_supported(int dk, int dv, int chunk_len);
+cudaError_t launch_seq(const FwdParams& p, cudaStream_t stream);
 cudaError_t static_scratch(void** ptr, size_t* bytes);
 int read_and_clear_device_status(cudaStream_t stream);
 void set_wait_limit_ns(uint64_t ns);
@@ -87,6 +89,7 @@ int to_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; 
 
 int run_bf16(const gdn::FwdParams& p, int chunk_len, cudaStream_t stream)
 {
+    if (p.T > 0 && gdn::seq_supported(p.dk, p.dv, chunk_len)) return to_status(gdn::launch_seq(p, stream));
     if (gdn::tc_supported(p.dk, p.dv, chunk_len)) return to_status(gdn::launch_tc(p, chunk_len, stream));
     return to_status(gdn::launch_ffma<__nv_bfloat16>(p, chunk_len, stream));
 }
@@ -479,6 +482,7 @@ int gdn_set_wait_limit_ns(unsigned long long ns)
 
 int gdn_bf16_path(int d_k, int d_v, int chunk_len)
 {
+    if (gdn::seq_supported(d_k, d_v, chunk_len)) return 2;
     return gdn::tc_supported(d_k, d_v, chunk_len) ? 1 : 0;
 }
 

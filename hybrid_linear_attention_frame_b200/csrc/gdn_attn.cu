@@ -423,13 +423,11 @@ cudaError_t launch_attn(const void* q, const void* k, const void* v, void* out, 
     if (!make_map_rows128(&mq, q, dk, H, T, B) || !make_map_rows128(&mk, k, dk, H, T, B) ||
         !make_map_rows128(&mv, v, dv, H, T, B))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(attn::chunk_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)attn::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    // the dynamic shared memory limit is a per-device setting of the current context: set it on
+    // every call (cheap), so that every device and a context re-created after a reset get it
+    cudaError_t e = cudaFuncSetAttribute(attn::chunk_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)attn::kSmemBytes);
+    if (e != cudaSuccess) return e;
     attn::AttnArgs a;
     a.out = out;
     a.B = B; a.H = H; a.T = T; a.dk = dk; a.dv = dv;

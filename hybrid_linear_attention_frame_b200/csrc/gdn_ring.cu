@@ -36,6 +36,8 @@
 // and the output, warps 14 and 15 load the two parts of the chain's slots.
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "gdn_common.cuh"
 #include "gdn_status.cuh"
 #include "gdn_sm100.cuh"
@@ -980,15 +982,13 @@ bool ring_supported(int dk, int dv, int chunk_len)
 // device: every CTA of the cooperative grid must be resident at once.
 cudaError_t ring_groups(int BH, int dv, int* groups)
 {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(ring::gdn_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)ring::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    // the dynamic shared memory limit is a per-device setting of the current context: set it on
+    // every call (cheap), so that every device and a context re-created after a reset get it
+    cudaError_t e = cudaFuncSetAttribute(ring::gdn_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)ring::kSmemBytes);
+    if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ring::gdn_ring_kernel, ring::kThreads,
@@ -1014,19 +1014,24 @@ static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 // Address of the static scratch on the current device, looked up once per
 // device (the first call on a device must not be inside a stream capture).
+// The cache is an atomic per device, so that threads making their first call
+// at the same time store the same value without a data race.  A device reset
+// (cudaDeviceReset) unloads the module: the cached address is then stale.
 cudaError_t static_scratch(void** ptr, size_t* bytes)
 {
     constexpr int kMaxDevices = 64;
-    static void* addr[kMaxDevices] = {};
+    static std::atomic<void*> addr[kMaxDevices] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    if (!addr[dev]) {
-        e = cudaGetSymbolAddress(&addr[dev], g_static_scratch);
+    void* a = addr[dev].load(std::memory_order_acquire);
+    if (!a) {
+        e = cudaGetSymbolAddress(&a, g_static_scratch);
         if (e != cudaSuccess) return e;
+        addr[dev].store(a, std::memory_order_release);
     }
-    *ptr = addr[dev];
+    *ptr = a;
     *bytes = kStaticScratchBytes;
     return cudaSuccess;
 }

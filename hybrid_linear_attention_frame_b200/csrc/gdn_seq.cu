@@ -1,0 +1,904 @@
+// Sequence-parallel chunked GDN forward for sm_100a: every SM runs the whole
+// per-chunk pipeline (prep, state chain, output) of its own stretch of chunks,
+// for all d_v state columns, with no communication between CTAs.
+//
+// Work split.  The B*H chains of N_c = ceil(T/64) chunks form one list of
+// units (chain-major).  CTA g takes the contiguous units [U g / G, U (g+1) / G):
+// at most the tail of one chain, some whole chains and the head of another.
+// A stretch that starts inside a chain needs the state entering its first
+// chunk.  The recurrence forgets geometrically: the homogeneous part of one
+// token step, a_t (I - b_t k^_t k^_t^T), has spectral norm <= a_t (the
+// normalised key has |k^| < 1 and b_t lies in (0, 1)), so the state entering
+// chunk c0 depends on the state entering an earlier chunk cw only through a
+// map of norm <= prod_{t in [64 cw, 64 c0)} a_t.  The CTA therefore starts the
+// recurrence from a zero state at the latest chunk cw < c0 at which that
+// product of gates has fallen to 2^-48 or below (outputs before c0 are not
+// written), or, when the gates never shrink that far, at the chain's first
+// chunk from the caller's initial state (then it runs the exact recurrence).
+// With the SANA-WM gates (a ~ 0.12 per token) one chunk of warm-up suffices.
+//
+// Per chunk of 64 tokens (notation of gdn_common.cuh; M = 128 everywhere by
+// stacking two 64-row operands, fp32 accumulators in TMEM):
+//   prep  Gram  [K;Q][K;Q]^T            -> norms (diagonal), A and P with the decay
+//         T = (I+A)^{-1} diag(beta), T' = T diag(e^G/|k|)  (CUDA cores + mma.sync)
+//         U = [Z;T] V, then W = [T';Z] K accumulated  -> EQS = [W ; U]
+//         -W to shared memory beside Q; lanes 0-63 of EQS cleared  -> EQS = [0 ; U]
+//   chain MMA1  [Q;-W] S_bf16 onto EQS   -> [Q S ; E = U - W S]
+//         E' = diag(e^{G_L-G}/|k|) E and E in bf16;  Q S scaled by e^G/|q| in TMEM
+//         MMA2  K^T E' onto SACC = e^{G_L} S  -> next state (fp32, in TMEM)
+//         PE    [P;X] E onto EQS lanes 0-63   -> O = diag(e^G/|q|) Q S + P E
+// The state lives in TMEM in fp32 and only its bf16 copy feeds MMA1.  When the
+// state is read back, the next chunk's decay e^{G_L} is applied to it, so that
+// MMA2 adds onto the already decayed state.
+//
+// Warp roles (16 warps): 0 loads q and k tiles (TMA), 1 issues the Gram MMAs,
+// 2 issues the chain MMAs, 3 issues the W/U MMAs and loads v tiles, 4-11 prep,
+// 12-15 chain and output.  Hand-offs are mbarriers; every wait is bounded and
+// gives up with GDN_ERR_TIMEOUT.
+#include <cooperative_groups.h>
+#include <cudaTypedefs.h>
+
+#include "gdn_common.cuh"
+#include "gdn_status.cuh"
+#include "gdn_sm100.cuh"
+
+namespace gdn {
+namespace seq {
+
+using namespace sm100;
+using tc::kC;
+using tc::kXS;
+
+constexpr int kThreads = 512;
+constexpr int kMaxAtoms = 7;                 // d_k, d_v <= 112 (16-column atoms)
+constexpr int kWarpLoadKQ = 0, kWarpGram = 1, kWarpChainMma = 2, kWarpWU = 3;
+constexpr int kPrepWarp0 = 4, kChainWarp0 = 12;
+constexpr int kPrepThreads = 256;
+constexpr uint32_t kBarPrep = 1;             // named barrier of the prep warps (3: the UT inverse's)
+
+// product of gates over a warm-up stretch below which the state entering it is dropped: 2^-48
+constexpr float kWarmupLogDecay = 48.0f * 0.693147181f;
+
+// TMEM columns (128 lanes each)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColG = 0;                // Gram [K;Q][K;Q]^T (N 128)
+constexpr uint32_t kColEQS = 128;            // 2 x 128: [W;U] -> [0;U] -> [QS;E] -> [O;-]
+constexpr uint32_t kColSacc = 384;           // state: d_k lanes x d_v columns
+
+// Shared memory (bytes from a 1024-aligned base).  d-indexed tiles are made of
+// 16-column atoms in the 32-byte swizzle (a row of an atom is 32 B, 16-byte
+// chunk c of row r at c ^ ((r >> 2) & 1)), so d = 112 wastes no space; the
+// 64 x 64 token tiles use the 128-byte swizzle.
+constexpr uint32_t kAtomKQW = 6144;          // per d_k atom: K rows | Q rows | W rows (64 each)
+constexpr uint32_t kAtQ = 2048, kAtW = 4096;
+constexpr uint32_t kStageSc = kMaxAtoms * kAtomKQW;          // chain scalars of the stage
+constexpr uint32_t kStageBytes = kStageSc + 1024;
+constexpr uint32_t kOffV = 2 * kStageBytes;                  // v tile, d_v atoms of 64 rows
+constexpr uint32_t kAtomV = 2048;
+constexpr uint32_t kTile = 8192;                             // 64 x 64 bf16, 128-byte swizzle
+constexpr uint32_t kOffP = kOffV + kMaxAtoms * kAtomV;       // P[2]; [P;X] reads the next 8 KB
+constexpr uint32_t kOffTp = kOffP + 2 * kTile;               // T' | Z | T
+constexpr uint32_t kOffZ = kOffTp + kTile;
+constexpr uint32_t kOffT = kOffZ + kTile;
+constexpr uint32_t kOffS = kOffT + kTile;                    // S bf16, d_v atoms of 112 rows
+constexpr uint32_t kAtomS = 112 * 32;
+constexpr uint32_t kOffEp = kOffS + kMaxAtoms * kAtomS;      // E' bf16, d_v atoms of 64 rows
+constexpr uint32_t kAtomE = 64 * 32;
+constexpr uint32_t kOffE = kOffEp + kMaxAtoms * kAtomE;      // E bf16
+constexpr uint32_t kOffAXI = kOffE + kMaxAtoms * kAtomE;     // fp32 [64][kXS]: A / (I+A)^{-1}
+constexpr uint32_t kScFloats = 13 * 64 + 16;
+constexpr uint32_t kOffSc = kOffAXI + 64 * kXS * 4;          // prep scalar table
+constexpr uint32_t kOffBar = kOffSc + kScFloats * 4;
+enum : uint32_t {
+    B_FULL = 0,       // [2] q/k tiles of a stage landed
+    B_SFREE = 2,      // [2] chain MMAs done with a stage (and with its P)
+    B_VFULL = 4,      // v tile landed
+    B_VFREE = 5,      // U MMA done with the v tile
+    B_G1 = 6,         // Gram done
+    B_GFREE = 7,      // Gram read by the prep
+    B_TREADY = 8,     // T' and T written
+    B_WU = 9,         // U and W MMAs done
+    B_READY = 10,     // [2] stage complete for the chain (-W written, EQS = [0;U], scalars)
+    B_EQFREE = 12,    // [2] output read from EQS
+    B_SREADY = 14,    // bf16 state written and SACC decayed
+    B_M1 = 15,        // MMA1 done
+    B_EREADY = 16,    // E' written
+    B_PEGO = 17,      // E written and Q S scaled
+    B_M2 = 18,        // MMA2 done
+    B_PEDONE = 19,    // P E done
+    kNumBars = 20,
+};
+constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+constexpr uint32_t kOffWarm = kOffAbort + 4;                 // warm-up start chunk of the first stretch
+constexpr uint32_t kSmemUsed = kOffWarm + 4;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;
+
+// prep scalar table (floats)
+enum : uint32_t {
+    SC_G = 0,        // cumulative log-gate G_i
+    SC_BETA = 64,    // beta_i (0 beyond the chunk)
+    SC_RK = 128,     // 1 / |k_i|
+    SC_RQ = 192,     // 1 / |q_i|
+    SC_GAM = 256,    // e^{G_i}
+    SC_DL = 320,     // e^{G_L - G_i} (0 beyond the chunk), times 1/|k_i| once the norms are known
+    SC_EXR = 384,    // e^{G_i - G_{16 floor(i/16) - 1}}   (i >= 16)
+    SC_EXC = 448,    // [4][64]: e^{G_{16 b - 1} - G_j}   (j < 16 b; row 0 unused)
+    SC_BGK = 704,    // beta_j e^{G_j} / |k_j|
+    SC_MISC = 768,
+};
+// chain scalars of a stage (floats): e^G/|q| and e^{G_L-G}/|k| (0 beyond the chunk)
+enum : uint32_t { CS_GQ = 0, CS_DL = 64 };
+
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffP % 1024 == 0 && kOffTp % 1024 == 0 && kStageBytes % 1024 == 0, "SW128 alignment");
+static_assert(kOffS % 256 == 0 && kOffEp % 256 == 0 && kOffE % 256 == 0 && kOffV % 256 == 0 &&
+                  kAtomKQW % 256 == 0 && kAtomS % 256 == 0,
+              "SW32 alignment");
+static_assert(4 * tc::kMS * 32 * 4 <= kTile, "solve scratch fits in the T tile");
+static_assert(kOffAXI % 16 == 0 && kOffSc % 16 == 0 && kOffBar % 8 == 0, "alignment");
+
+constexpr uint32_t kIdGram = idesc_bf16(128, 128, false, false);
+
+__host__ __device__ constexpr uint32_t bar_count(uint32_t i) {
+    return (i == B_SREADY || i == B_PEGO) ? 4u : (i == B_EQFREE || i == B_EQFREE + 1 || i == B_EREADY) ? 2u : 1u;
+}
+
+// descriptors: K-major / MN-major 32-byte swizzle (8-row groups 256 B apart), K-major 128-byte swizzle
+__device__ __forceinline__ uint64_t dk32(uint32_t a) { return smem_desc(a, 16, 256, kSwizzle32); }
+__device__ __forceinline__ uint64_t dmn32(uint32_t a, uint32_t lbo) { return smem_desc(a, lbo, 256, kSwizzle32); }
+__device__ __forceinline__ uint64_t dk128(uint32_t a) { return smem_desc(a, 16, 1024, kSwizzle128); }
+
+__device__ __forceinline__ uint32_t tlane(uint32_t tmem, int quarter) {
+    return tmem + ((uint32_t)(32 * quarter) << 16);
+}
+
+// Shared address of the 8 columns [c8, c8 + 8) of row r in a tile of SW32 atoms `lbo` bytes apart.
+__device__ __forceinline__ uint32_t sw32_at(uint32_t tile, uint32_t lbo, uint32_t r, uint32_t c8) {
+    return tile + (c8 >> 4) * lbo + sw32_chunk_offset(r, (c8 >> 3) & 1u);
+}
+
+__device__ __forceinline__ void st_bf16x8(uint32_t addr, const float* x) {
+    st_shared_v4(addr, pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                 pack_bf16x2(x[6], x[7]));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32"
+                 " [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 :: "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+                    "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+                    "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+                    "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+                    "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+                    "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float softplus_fast(float x) { return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x))); }
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+__device__ __forceinline__ bool group_all(uint32_t id, uint32_t n, bool v) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.u32 p, %3, 0;\n\t"
+                 "bar.red.and.pred q, %1, %2, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"(id), "r"(n), "r"(v ? 1u : 0u) : "memory");
+    return r != 0;
+}
+
+struct SeqArgs {
+    FwdParams p;
+    uint64_t wait_limit_ns;
+    int G;            // CTAs
+    int grid_sync;    // state_in aliases state_out: every read of it precedes every write
+};
+
+// ---------------------------------------------------------------- work split
+
+// This CTA's stretch [u0, u1) of units x * nc + c, as pieces of consecutive
+// chains ("range order"): piece 0 starts at chunk c0 of chain x0, every later
+// piece at chunk 0; the last one ends at chunk cl.
+struct Plan {
+    int nc, x0, c0, np, cl;
+    int head_first;   // the last piece starts at chunk 0 and stops inside its chain: run it first
+};
+
+__device__ __forceinline__ Plan make_plan(const SeqArgs& a) {
+    Plan P;
+    const int nc = (a.p.T + kC - 1) / kC;
+    const long long U = (long long)a.p.B * a.p.H * nc;
+    const long long u0 = U * blockIdx.x / a.G, u1 = U * (blockIdx.x + 1) / a.G;
+    P.nc = nc;
+    P.x0 = (int)(u0 / nc);
+    P.c0 = (int)(u0 - (long long)P.x0 * nc);
+    const int xl = (int)((u1 - 1) / nc);
+    P.np = xl - P.x0 + 1;
+    P.cl = (int)(u1 - 1 - (long long)xl * nc) + 1;
+    P.head_first = (P.np > 1 && P.cl < nc) ? 1 : 0;
+    return P;
+}
+
+struct Piece {
+    int b, h, cw, c0, c1;   // chain (b, h); chunks [cw, c1) run, outputs from c0 on
+    bool rd, wr;            // starts from state_in / ends the chain and writes state_out
+};
+
+// Pieces in processing order: the head of a chain (whose state another CTA
+// writes at the chain's end) first, so that every read of an initial state by
+// a CTA that does not also write that chain's final state happens at the start.
+__device__ __forceinline__ Piece piece_at(const SeqArgs& a, const Plan& P, int k, int warm0) {
+    int j = k;
+    if (P.head_first) j = (k == 0) ? P.np - 1 : k - 1;
+    Piece pc;
+    const int x = P.x0 + j;
+    pc.b = x / a.p.H;
+    pc.h = x - pc.b * a.p.H;
+    pc.c0 = (j == 0) ? P.c0 : 0;
+    pc.c1 = (j == P.np - 1) ? P.cl : P.nc;
+    pc.cw = (j == 0) ? warm0 : 0;
+    pc.rd = pc.cw == 0 && a.p.state_in != nullptr;
+    pc.wr = pc.c1 == P.nc && a.p.state_out != nullptr;
+    return pc;
+}
+
+// Cursor over the chunks this CTA runs, in processing order (n counts them).
+struct Cursor {
+    const SeqArgs* a;
+    const Plan* P;
+    int warm0, k, c, n;
+    Piece pc;
+    __device__ __forceinline__ Cursor(const SeqArgs& a_, const Plan& P_, int warm0_)
+        : a(&a_), P(&P_), warm0(warm0_), k(0), c(0), n(0) {
+        pc = piece_at(*a, *P, 0, warm0);
+        c = pc.cw;
+    }
+    __device__ __forceinline__ bool valid() const { return k < P->np; }
+    __device__ __forceinline__ bool first() const { return c == pc.cw; }
+    __device__ __forceinline__ bool last() const { return c == pc.c1 - 1; }
+    __device__ __forceinline__ int L() const { return min(kC, a->p.T - c * kC); }
+    __device__ __forceinline__ void next() {
+        ++n;
+        if (++c >= pc.c1) {
+            if (++k < P->np) {
+                pc = piece_at(*a, *P, k, warm0);
+                c = pc.cw;
+            }
+        }
+    }
+};
+
+// Sum over the tokens of chunk c of chain (b, h) of -log a_t (whole warp; all lanes get it).
+__device__ __forceinline__ float chunk_decay(const FwdParams& p, int b, int h, int c, int lane) {
+    float s = 0.0f;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int t = c * kC + lane + 32 * r;
+        if (t < p.T && gate_applies(p, t))
+            s += softplus_fast(__ldg(p.gate + ((size_t)b * p.F + t / p.frame_len) * p.H + h));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    return s;
+}
+
+// ---------------------------------------------------------------- the kernel
+
+__global__ void __launch_bounds__(kThreads, 1)
+gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const SeqArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gb = smem_raw + (base - raw);
+    const FwdParams& p = a.p;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, qtr = warp & 3;
+    const int dk = p.dk, dv = p.dv, nak = dk / 16, nav = dv / 16;
+    const uint64_t lim = a.wait_limit_ns;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + kOffAbort);
+    auto bar = [&](uint32_t i) { return base + kOffBar + 8u * i; };
+    const Plan P = make_plan(a);
+
+    if (warp == 0) {
+        tmem_alloc(base + kOffTmemSlot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 32) {
+        for (uint32_t i = 0; i < kNumBars; ++i) mbar_init(bar(i), bar_count(i));
+        fence_mbar_init();
+        *abort_flag = 0;
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == kWarpWU) {
+        // warm-up start of the first piece (see the file comment)
+        int cw = P.c0;
+        if (P.c0 > 0) {
+            const int b = P.x0 / p.H, h = P.x0 - (P.x0 / p.H) * p.H;
+            float acc = 0.0f;
+            cw = 0;
+            for (int c = P.c0 - 1; c >= 0; --c) {
+                acc += chunk_decay(p, b, h, c, lane);
+                if (acc >= kWarmupLogDecay) {
+                    cw = c;
+                    break;
+                }
+            }
+        }
+        if (lane == 0) *reinterpret_cast<volatile int*>(gb + kOffWarm) = cw;
+    }
+    // the zero tile Z
+    for (int i = tid; i < (int)(kTile / 16); i += kThreads) st_shared_v4(base + kOffZ + 16u * i, 0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gb + kOffTmemSlot);
+    const int warm0 = *reinterpret_cast<volatile int*>(gb + kOffWarm);
+
+    // Chain warps: S tile and SACC for the first chunk of a piece (state_in or zero),
+    // then SREADY.  SACC holds e^{G_L} S for the chunk about to run.
+    auto chain_init = [&](const Piece& pc) {
+        const int q = warp - kChainWarp0, row = 32 * q + lane;
+        const float gl = __expf(-chunk_decay(p, pc.b, pc.h, pc.cw, lane));
+        const float* si = (pc.rd && row < dk)
+                              ? p.state_in + (((size_t)pc.b * p.H + pc.h) * dk + row) * (size_t)dv
+                              : nullptr;
+        for (int at = 0; at < nav; ++at) {
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+            if (si) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 f = *reinterpret_cast<const float4*>(si + 16 * at + 4 * j);
+                    v[4 * j] = f.x; v[4 * j + 1] = f.y; v[4 * j + 2] = f.z; v[4 * j + 3] = f.w;
+                }
+            }
+            if (row < dk) {
+                st_bf16x8(sw32_at(base + kOffS, kAtomS, row, 16 * at), v);
+                st_bf16x8(sw32_at(base + kOffS, kAtomS, row, 16 * at + 8), v + 8);
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] *= gl;
+            tmem_st16(tlane(tmem + kColSacc, q) + 16u * at, v);
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_SREADY));
+    };
+    if (warp >= kChainWarp0 && P.np > 0) chain_init(piece_at(a, P, 0, warm0));
+    if (a.grid_sync) {
+        // in-place state: every CTA has read the initial states it needs before any final state is written
+        tc_fence_before();
+        cooperative_groups::this_grid().sync();
+        tc_fence_after();
+    }
+
+    if (warp == kWarpLoadKQ) {
+        // ======================= q and k tiles (TMA) =======================
+        bool ok = true;
+        int issued = 0;
+        for (Cursor cu(a, P, warm0); cu.valid(); cu.next()) {
+            const int n = cu.n, s = n & 1;
+            if (n >= 2) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFREE + s), (uint32_t)(((n - 2) >> 1) & 1),
+                                                       abort_flag, lim, 21));
+                if (!ok) break;
+            }
+            if (lane == 0) {
+                const uint32_t st = base + (uint32_t)s * kStageBytes, fb = bar(B_FULL + s);
+                mbar_arrive_expect_tx(fb, (uint32_t)nak * 2u * 2048u);
+                for (int at = 0; at < nak; ++at) {
+                    tma_load_4d(st + (uint32_t)at * kAtomKQW, &tm_k, fb, 16 * at, cu.pc.h, cu.c * kC, cu.pc.b);
+                    tma_load_4d(st + (uint32_t)at * kAtomKQW + kAtQ, &tm_q, fb, 16 * at, cu.pc.h, cu.c * kC,
+                                cu.pc.b);
+                }
+            }
+            __syncwarp();
+            issued = n + 1;
+        }
+        if (!ok && lane == 0)
+            for (int m = max(0, issued - 2); m < issued; ++m)
+                drain_wait(bar(B_FULL + (m & 1)), (uint32_t)((m >> 1) & 1));
+        __syncwarp();
+    } else if (warp == kWarpGram) {
+        // ======================= Gram MMAs =======================
+        bool ok = true;
+        int issued = 0;
+        for (Cursor cu(a, P, warm0); cu.valid(); cu.next()) {
+            const int n = cu.n, s = n & 1;
+            ok = mbar_wait(bar(B_FULL + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 22);
+            if (ok && n > 0) ok = mbar_wait(bar(B_GFREE), (uint32_t)((n - 1) & 1), abort_flag, lim, 23);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t st = base + (uint32_t)s * kStageBytes;
+#pragma unroll 1
+            for (int at = 0; at < nak; ++at) {
+                const uint64_t d = dk32(st + (uint32_t)at * kAtomKQW);
+                mma_bf16_warp(tmem + kColG, d, d, kIdGram, at > 0);
+            }
+            mma_commit_warp(bar(B_G1));
+            issued = n + 1;
+        }
+        if (!ok && issued > 0 && lane == 0) drain_wait(bar(B_G1), (uint32_t)((issued - 1) & 1));
+        __syncwarp();
+    } else if (warp == kWarpWU) {
+        // ======================= U and W MMAs; v tiles =======================
+        const uint32_t idu = idesc_bf16(128, dv, false, true), idw = idesc_bf16(128, dk, false, true);
+        bool ok = true;
+        int v_issued = 0, wu_issued = 0;
+        Cursor cv(a, P, warm0);
+        auto load_v = [&](const Cursor& c) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(B_VFULL), (uint32_t)nav * 2048u);
+                for (int at = 0; at < nav; ++at)
+                    tma_load_4d(base + kOffV + (uint32_t)at * kAtomV, &tm_v, bar(B_VFULL), 16 * at, c.pc.h, c.c * kC,
+                                c.pc.b);
+            }
+            __syncwarp();
+        };
+        if (cv.valid()) {
+            load_v(cv);
+            v_issued = 1;
+        }
+        for (Cursor cu(a, P, warm0); cu.valid(); cu.next()) {
+            const int n = cu.n, s = n & 1;
+            const uint32_t eqs = tmem + kColEQS + 128u * (uint32_t)s;
+            ok = mbar_wait(bar(B_TREADY), (uint32_t)(n & 1), abort_flag, lim, 24);
+            ok = ok && mbar_wait(bar(B_VFULL), (uint32_t)(n & 1), abort_flag, lim, 25);
+            if (ok && n >= 2) ok = mbar_wait(bar(B_EQFREE + s), (uint32_t)(((n - 2) >> 1) & 1), abort_flag, lim, 26);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t st = base + (uint32_t)s * kStageBytes;
+#pragma unroll
+            for (int ks = 0; ks < kC / 16; ++ks)   // [Z;T] V -> [0 ; U]
+                mma_bf16_warp(eqs, dk128(base + kOffZ + 32u * ks), dmn32(base + kOffV + 512u * ks, kAtomV), idu,
+                              ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < kC / 16; ++ks)   // + [T';Z] K -> [W ; U]
+                mma_bf16_warp(eqs, dk128(base + kOffTp + 32u * ks), dmn32(st + 512u * ks, kAtomKQW), idw, 1u);
+            mma_commit_warp(bar(B_WU));
+            mma_commit_warp(bar(B_VFREE));
+            wu_issued = n + 1;
+            cv.next();
+            if (cv.valid()) {
+                // the next chunk's v tile, once this U MMA has read the buffer
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_VFREE), (uint32_t)(n & 1), abort_flag, lim, 27));
+                if (!ok) break;
+                load_v(cv);
+                v_issued = n + 2;
+            }
+        }
+        if (!ok && lane == 0) {
+            if (wu_issued > 0) drain_wait(bar(B_WU), (uint32_t)((wu_issued - 1) & 1));
+            if (v_issued > wu_issued) drain_wait(bar(B_VFULL), (uint32_t)((v_issued - 1) & 1));
+        }
+        __syncwarp();
+    } else if (warp == kWarpChainMma) {
+        // ======================= chain MMAs =======================
+        const uint32_t id1 = idesc_bf16(128, dv, false, true), id2 = idesc_bf16(128, dv, true, true);
+        bool ok = true;
+        int pending = -1, pend_n = 0;
+        for (Cursor cu(a, P, warm0); cu.valid(); cu.next()) {
+            const int n = cu.n, s = n & 1;
+            const uint32_t eqs = tmem + kColEQS + 128u * (uint32_t)s;
+            const uint32_t st = base + (uint32_t)s * kStageBytes;
+            ok = mbar_wait(bar(B_READY + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 31);
+            ok = ok && mbar_wait(bar(B_SREADY), (uint32_t)(n & 1), abort_flag, lim, 32);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll 1
+            for (int at = 0; at < nak; ++at)       // [Q;-W] S onto [0 ; U]
+                mma_bf16_warp(eqs, dk32(st + (uint32_t)at * kAtomKQW + kAtQ), dmn32(base + kOffS + 512u * at, kAtomS),
+                              id1, 1u);
+            mma_commit_warp(bar(B_M1));
+            pending = B_M1; pend_n = n;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_EREADY), (uint32_t)(n & 1), abort_flag, lim, 33));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < kC / 16; ++ks)    // K^T E' onto e^{G_L} S
+                mma_bf16_warp(tmem + kColSacc, dmn32(st + 512u * ks, kAtomKQW), dmn32(base + kOffEp + 512u * ks, kAtomE),
+                              id2, 1u);
+            mma_commit_warp(bar(B_M2));
+            pending = B_M2;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEGO), (uint32_t)(n & 1), abort_flag, lim, 34));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t pa = base + kOffP + kTile * (uint32_t)s;
+#pragma unroll
+            for (int ks = 0; ks < kC / 16; ++ks)    // [P;X] E onto [(e^G/|q|) Q S ; -]
+                mma_bf16_warp(eqs, dk128(pa + 32u * ks), dmn32(base + kOffE + 512u * ks, kAtomE), id1, 1u);
+            mma_commit_warp(bar(B_PEDONE));
+            mma_commit_warp(bar(B_SFREE + s));
+            pending = B_PEDONE;
+        }
+        if (!ok && pending >= 0 && lane == 0) drain_wait(bar((uint32_t)pending), (uint32_t)(pend_n & 1));
+        __syncwarp();
+    } else if (warp < kChainWarp0) {
+        // ======================= prep (warps 4-11) =======================
+        const int pt = tid - kPrepWarp0 * 32, pw = warp - kPrepWarp0;
+        float* sc = reinterpret_cast<float*>(gb + kOffSc);
+        float* AXI = reinterpret_cast<float*>(gb + kOffAXI);
+        float* MSf = reinterpret_cast<float*>(gb + kOffT);
+        const uint32_t tg = tmem + kColG;
+        bool ok = true;
+        // gate and beta logits of the next chunk, loaded one chunk ahead (warp pw 0)
+        float pg0 = 0.f, pg1 = 0.f, pb0 = 0.f, pb1 = 0.f;
+        auto load_logits = [&](const Cursor& c) {
+            const int L = c.L(), i0 = 2 * lane, t0 = c.c * kC + i0;
+            pg0 = pg1 = pb0 = pb1 = 0.0f;
+            if (i0 < L) {
+                pg0 = __ldg(p.gate + ((size_t)c.pc.b * p.F + t0 / p.frame_len) * p.H + c.pc.h);
+                pb0 = __ldg(p.beta + ((size_t)c.pc.b * p.T + t0) * p.H + c.pc.h);
+            }
+            if (i0 + 1 < L) {
+                pg1 = __ldg(p.gate + ((size_t)c.pc.b * p.F + (t0 + 1) / p.frame_len) * p.H + c.pc.h);
+                pb1 = __ldg(p.beta + ((size_t)c.pc.b * p.T + t0 + 1) * p.H + c.pc.h);
+            }
+        };
+        Cursor cn(a, P, warm0);
+        if (pw == 0 && cn.valid()) load_logits(cn);
+        for (Cursor cu(a, P, warm0); cu.valid(); cu.next()) {
+            const int n = cu.n, s = n & 1, L = cu.L();
+            float* cs = reinterpret_cast<float*>(gb + (uint32_t)s * kStageBytes + kStageSc);
+            const uint32_t stg = base + (uint32_t)s * kStageBytes;
+            // ---- gates: G (warp scan), beta; then the decay tables ----
+            if (pw == 0) {
+                const int i0 = 2 * lane, t0 = cu.c * kC + i0;
+                const float la0 = (i0 < L && gate_applies(p, t0)) ? -softplus_fast(pg0) : 0.0f;
+                const float la1 = (i0 + 1 < L && gate_applies(p, t0 + 1)) ? -softplus_fast(pg1) : 0.0f;
+                float x = la0 + la1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                sc[SC_G + i0] = x - la1;
+                sc[SC_G + i0 + 1] = x;
+                sc[SC_BETA + i0] = (i0 < L) ? sigmoid_fast(pb0) : 0.0f;
+                sc[SC_BETA + i0 + 1] = (i0 + 1 < L) ? sigmoid_fast(pb1) : 0.0f;
+                cn.next();
+                if (cn.valid()) load_logits(cn);
+            }
+            named_bar_sync(kBarPrep, kPrepThreads);
+            {
+                const float GL = sc[SC_G + 63];
+                const int idx = pt;
+                if (idx < 64) {
+                    const int i = idx;
+                    const float Gi = sc[SC_G + i];
+                    sc[SC_GAM + i] = __expf(Gi);
+                    sc[SC_DL + i] = (i < L) ? __expf(GL - Gi) : 0.0f;
+                    sc[SC_EXR + i] = (i >= 16) ? __expf(Gi - sc[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
+                } else {
+                    const int bi = 1 + (idx - 64) / 64, j = idx & 63;
+                    sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? __expf(sc[SC_G + 16 * bi - 1] - sc[SC_G + j]) : 0.0f;
+                }
+            }
+            // ---- Gram done (this vote is also the barrier after the tables) ----
+            ok = mbar_wait(bar(B_G1), (uint32_t)(n & 1), abort_flag, lim, 41);
+            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            tc_fence_after();
+            // ---- norms from the Gram diagonal: |k_i|^2 (lanes 0-63), |q_i|^2 (lanes 64-127) ----
+            if (pw < 4) {
+                float v[32];
+                tmem_ld16(tlane(tg, qtr) + 32u * qtr, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_ld16(tlane(tg, qtr) + 32u * qtr + 16u, *reinterpret_cast<float(*)[16]>(&v[16]));
+                tmem_wait_ld();
+                float d = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) d = (j == lane) ? v[j] : d;
+                const float r = rsqrtf(d + kNormEps);
+                const int i = 32 * (qtr & 1) + lane;
+                if (qtr < 2) {
+                    sc[SC_RK + i] = r;
+                    const float dl = sc[SC_DL + i] * r;
+                    sc[SC_DL + i] = dl;
+                    cs[CS_DL + i] = dl;
+                    sc[SC_BGK + i] = sc[SC_BETA + i] * sc[SC_GAM + i] * r;
+                } else {
+                    sc[SC_RQ + i] = r;
+                    cs[CS_GQ + i] = r * sc[SC_GAM + i];
+                }
+            }
+            named_bar_sync(kBarPrep, kPrepThreads);
+            // ---- A (fp32, transposed above the diagonal of AXI) and P (bf16 tile P[s]) ----
+            {
+                const uint32_t ptile = base + kOffP + kTile * (uint32_t)s;
+                const int ch = pw >> 2;
+                if ((qtr & 1) == 0 && ch == 1) {
+                    // rows 0-31 x columns 32-63 lie above the diagonal: A has nothing there, P is zero
+                    if (qtr == 2) {
+                        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int g8 = 0; g8 < 4; ++g8) st_bf16x8(ptile + sw128_offset((uint32_t)lane, 32u + 8u * g8), z);
+                    }
+                } else {
+                    const int i = 32 * (qtr & 1) + lane;
+                    const int bi = i >> 4;
+                    const float Gi = sc[SC_G + i], exr = sc[SC_EXR + i];
+                    const float ri = (qtr < 2) ? sc[SC_BETA + i] * sc[SC_RK + i] : sc[SC_RQ + i];
+#pragma unroll 1
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int j0 = 32 * ch + 16 * hh;
+                        float v[16], val[16];
+                        tmem_ld16(tlane(tg, qtr) + (uint32_t)j0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 g4 = ld4(sc + SC_G + j0 + 4 * q4);
+                            const float4 r4 = ld4(sc + SC_RK + j0 + 4 * q4);
+                            const float4 e4 = ld4(sc + SC_EXC + 64 * bi + j0 + 4 * q4);
+                            const float gj[4] = {g4.x, g4.y, g4.z, g4.w};
+                            const float rkj[4] = {r4.x, r4.y, r4.z, r4.w};
+                            const float ex[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int jj = 4 * q4 + e, j = j0 + jj;
+                                const float dec = ((j >> 4) == bi) ? __expf(Gi - gj[e]) : exr * ex[e];
+                                const bool keep = (qtr < 2) ? (j < i) : (j <= i);
+                                val[jj] = keep ? ri * rkj[e] * v[jj] * dec : 0.0f;
+                            }
+                        }
+                        if (qtr < 2) {
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj)
+                                if (j0 + jj < i) AXI[(j0 + jj) * kXS + i] = val[jj];
+                        } else {
+                            st_bf16x8(ptile + sw128_offset((uint32_t)i, (uint32_t)j0), &val[0]);
+                            st_bf16x8(ptile + sw128_offset((uint32_t)i, (uint32_t)j0 + 8u), &val[8]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            if (pt == 0) mbar_arrive(bar(B_GFREE));       // the Gram accumulator may be overwritten
+            // ---- (I + A)^{-1} (warps 4-7) ----
+            if (pw < 4) tc::unit_lower_inverse_64(AXI, MSf, pt);
+            named_bar_sync(kBarPrep, kPrepThreads);
+            // ---- T = (I+A)^{-1} diag(beta), T' = T diag(beta e^G / |k|): bf16 tiles ----
+            {
+                const int i = pt >> 2, jb = 16 * (pt & 3);
+                float tv[16], tpv[16];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 x4 = ld4(AXI + i * kXS + jb + 4 * q4);
+                    const float4 b4 = ld4(sc + SC_BETA + jb + 4 * q4);
+                    const float4 f4 = ld4(sc + SC_BGK + jb + 4 * q4);
+                    const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+                    const float bs[4] = {b4.x, b4.y, b4.z, b4.w};
+                    const float fs[4] = {f4.x, f4.y, f4.z, f4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float x = (jb + 4 * q4 + e <= i) ? xs[e] : 0.0f;
+                        tv[4 * q4 + e] = x * bs[e];
+                        tpv[4 * q4 + e] = x * fs[e];
+                    }
+                }
+                st_bf16x8(base + kOffT + sw128_offset((uint32_t)i, (uint32_t)jb), &tv[0]);
+                st_bf16x8(base + kOffT + sw128_offset((uint32_t)i, (uint32_t)jb + 8u), &tv[8]);
+                st_bf16x8(base + kOffTp + sw128_offset((uint32_t)i, (uint32_t)jb), &tpv[0]);
+                st_bf16x8(base + kOffTp + sw128_offset((uint32_t)i, (uint32_t)jb + 8u), &tpv[8]);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            if (pt == 0) mbar_arrive(bar(B_TREADY));
+            // ---- U and W done: -W beside Q, then clear lanes 0-63 of EQS ----
+            ok = mbar_wait(bar(B_WU), (uint32_t)(n & 1), abort_flag, lim, 42);
+            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            tc_fence_after();
+            if (qtr < 2) {
+                const int i = 32 * qtr + lane;
+                const uint32_t eq = tlane(tmem + kColEQS + 128u * (uint32_t)s, qtr);
+                const int a0 = (pw < 4) ? 0 : 4, a1 = min(nak, a0 + 4);
+                for (int at = a0; at < a1; ++at) {
+                    float v[16];
+                    tmem_ld16(eq + 16u * at, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = -v[j];
+                    const uint32_t wa = stg + (uint32_t)at * kAtomKQW + kAtW;
+                    st_bf16x8(wa + sw32_chunk_offset((uint32_t)i, 0), &v[0]);
+                    st_bf16x8(wa + sw32_chunk_offset((uint32_t)i, 1), &v[8]);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+                    tmem_st16(eq + 16u * at, v);
+                }
+                tmem_wait_st();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            if (pt == 0) mbar_arrive(bar(B_READY + s));
+        }
+    } else {
+        // ======================= chain and output (warps 12-15) =======================
+        const int q = warp - kChainWarp0, row = 32 * q + lane;
+        bool ok = true;
+        for (Cursor cu(a, P, warm0); cu.valid(); cu.next()) {
+            const int n = cu.n, s = n & 1, L = cu.L();
+            const Piece& pc = cu.pc;
+            const bool last = cu.last(), emit = cu.c >= pc.c0;
+            if (cu.first() && n > 0) chain_init(pc);
+            const uint32_t eqs = tlane(tmem + kColEQS + 128u * (uint32_t)s, q);
+            const float* cs = reinterpret_cast<const float*>(gb + (uint32_t)s * kStageBytes + kStageSc);
+            // decay of the next chunk of this piece, applied to the state when it is read back
+            const float gl_next = last ? 1.0f : __expf(-chunk_decay(p, pc.b, pc.h, cu.c + 1, lane));
+            ok = mbar_wait(bar(B_READY + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 51);
+            ok = ok && mbar_wait(bar(B_M1), (uint32_t)(n & 1), abort_flag, lim, 52);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            if (q >= 2) {
+                // E (TMEM lanes 64-127): E' = diag(e^{G_L-G}/|k|) E for MMA2, then E for P E
+                const int i = row - 64;
+                const float dl = cs[CS_DL + i];
+                for (int at = 0; at < nav; ++at) {
+                    float v[16];
+                    tmem_ld16(eqs + 16u * at, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] *= dl;
+                    st_bf16x8(sw32_at(base + kOffEp, kAtomE, (uint32_t)i, 16u * at), &v[0]);
+                    st_bf16x8(sw32_at(base + kOffEp, kAtomE, (uint32_t)i, 16u * at + 8u), &v[8]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_EREADY));
+                for (int at = 0; at < nav; ++at) {
+                    float v[16];
+                    tmem_ld16(eqs + 16u * at, v);
+                    tmem_wait_ld();
+                    st_bf16x8(sw32_at(base + kOffE, kAtomE, (uint32_t)i, 16u * at), &v[0]);
+                    st_bf16x8(sw32_at(base + kOffE, kAtomE, (uint32_t)i, 16u * at + 8u), &v[8]);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_PEGO));
+            } else {
+                // Q S (TMEM lanes 0-63) scaled in place by e^G/|q|; P E is added onto it
+                const float gq = cs[CS_GQ + row];
+                for (int at = 0; at < nav; ++at) {
+                    float v[16];
+                    tmem_ld16(eqs + 16u * at, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] *= gq;
+                    tmem_st16(eqs + 16u * at, v);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_PEGO));
+            }
+            // ---- next state: bf16 copy for MMA1, decayed fp32 back into SACC ----
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_M2), (uint32_t)(n & 1), abort_flag, lim, 53));
+            if (!ok) break;
+            tc_fence_after();
+            {
+                const uint32_t sa = tlane(tmem + kColSacc, q);
+                float* so = (last && pc.wr && row < dk)
+                                ? p.state_out + (((size_t)pc.b * p.H + pc.h) * dk + row) * (size_t)dv
+                                : nullptr;
+                for (int at = 0; at < nav; ++at) {
+                    float v[16];
+                    tmem_ld16(sa + 16u * at, v);
+                    tmem_wait_ld();
+                    if (so) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<float4*>(so + 16 * at + 4 * j) =
+                                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    }
+                    if (!last) {
+                        if (row < dk) {
+                            st_bf16x8(sw32_at(base + kOffS, kAtomS, (uint32_t)row, 16u * at), &v[0]);
+                            st_bf16x8(sw32_at(base + kOffS, kAtomS, (uint32_t)row, 16u * at + 8u), &v[8]);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) v[j] *= gl_next;
+                        tmem_st16(sa + 16u * at, v);
+                    }
+                }
+                if (!last) {
+                    tmem_wait_st();
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(B_SREADY));
+                }
+            }
+            // ---- output rows (TMEM lanes 0-63) ----
+            if (q < 2) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEDONE), (uint32_t)(n & 1), abort_flag, lim, 54));
+                if (!ok) break;
+                tc_fence_after();
+                if (emit && p.out) {
+                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) +
+                                       (((size_t)pc.b * p.T + (size_t)cu.c * kC + row) * p.H + pc.h) * dv;
+                    for (int at = 0; at < nav; ++at) {
+                        float v[16];
+                        tmem_ld16(eqs + 16u * at, v);
+                        tmem_wait_ld();
+                        if (row < L) {
+                            uint4* o4 = reinterpret_cast<uint4*>(o + 16 * at);
+                            o4[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                               pack_bf16x2(v[6], v[7]));
+                            o4[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                                               pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_EQFREE + s));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace seq
+
+// ---------------------------------------------------------------- host side
+
+bool seq_supported(int dk, int dv, int chunk_len)
+{
+    return chunk_len == seq::kC && dk % 16 == 0 && dv % 16 == 0 && dk >= 16 && dv >= 16 &&
+           dk <= 16 * seq::kMaxAtoms && dv <= 16 * seq::kMaxAtoms;
+}
+
+cudaError_t launch_seq(const FwdParams& p, cudaStream_t stream)
+{
+    if (!seq_supported(p.dk, p.dv, seq::kC) || p.T < 1) return cudaErrorInvalidValue;
+    // the dynamic shared memory limit is a per-device setting of the current context: set it on
+    // every call (cheap), so that every device and a context re-created after a reset get it
+    cudaError_t e = cudaFuncSetAttribute(seq::gdn_seq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)seq::kSmemBytes);
+    int dev = 0, sms = 0;
+    if (e == cudaSuccess) e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long nc = (p.T + seq::kC - 1) / seq::kC;
+    const long long U = (long long)p.B * p.H * nc;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, p.q, p.dk, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+        !make_map(&mk, p.k, p.dk, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+        !make_map(&mv, p.v, p.dv, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B))
+        return cudaErrorInvalidValue;
+    seq::SeqArgs args;
+    args.p = p;
+    args.wait_limit_ns = g_wait_limit_ns;
+    args.G = (int)(U < sms ? U : sms);
+    args.grid_sync = (p.state_in != nullptr && (const void*)p.state_in == (const void*)p.state_out) ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)args.G);
+    cfg.blockDim = dim3(seq::kThreads);
+    cfg.dynamicSmemBytes = seq::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = args.grid_sync ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, seq::gdn_seq_kernel, mq, mk, mv, args);
+}
+
+}  // namespace gdn

@@ -83,12 +83,16 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
 // (first error wins) and returns false.
 // (The polling loop is an out-of-line function: waits are many and mostly
 // succeed at once, and inlining the loop everywhere bloats the code.)
+// Under a short bound (below 1 ms) the phase is polled without the suspend
+// hint and the clock read at every poll, so that the bound is observed even
+// when the phase completes within the hint's time.
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
                                             uint64_t limit_ns, int code) {
     const uint64_t t0 = globaltimer_ns();
+    const bool short_bound = limit_ns < 1000000ull;
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait_hint(bar, parity, 1000u)) return true;
-        if ((it & 63u) == 0) {
+        if (short_bound ? mbar_try_wait(bar, parity) : mbar_try_wait_hint(bar, parity, 1000u)) return true;
+        if (short_bound || (it & 63u) == 0) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
                 *abort = 1;

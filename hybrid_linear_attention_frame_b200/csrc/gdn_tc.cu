@@ -851,14 +851,11 @@ cudaError_t launch_tc(const FwdParams& p, int chunk_len, cudaStream_t stream)
         !make_map(&mk, p.k, p.dk, p.H, T, p.B, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mv, p.v, p.dv, p.H, T, p.B, tc::kVB, CU_TENSOR_MAP_SWIZZLE_32B))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc::gdn_chunk_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)tc::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    // the dynamic shared memory limit is a per-device setting of the current context: set it on
+    // every call (cheap), so that every device and a context re-created after a reset get it
+    cudaError_t e = cudaFuncSetAttribute(tc::gdn_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tc::kSmemBytes);
+    if (e != cudaSuccess) return e;
     tc::TcArgs args;
     args.p = p;
     args.wait_limit_ns = g_wait_limit_ns;

@@ -78,6 +78,23 @@ typedef enum {
  *   state_in   may be NULL: zero initial state.
  *   state_out  may be NULL: the final state is not written.
  * Returns a gdn_status.
+ *
+ * Which kernel runs (gdn_bf16_path reports it).  With chunk_len 64 and
+ * d_k, d_v <= 112 (the SANA-WM layer has 112): the sequence-parallel kernel,
+ * the fast path, with no workspace.  Every SM runs the whole per-chunk pipeline
+ * of its own stretch of the B*H chains' chunks.  A stretch that begins inside a
+ * chain starts the recurrence from a zero state at the latest earlier chunk
+ * past which the product of the gates a_t has fallen to 2^-48 or below; where
+ * the gates never shrink that far, it starts at the chain's first token from
+ * state_in.  The state dropped that way is damped by the gates to 2^-48 of its
+ * size: a bound, not an estimate, since a token step without its write has
+ * spectral norm <= a_t.  So the result equals the recurrence up to rounding.
+ * Slowly decaying gates make those warm-ups longer and the call slower, down
+ * to one SM per chain when nothing decays.  With d_k or d_v = 128: a kernel
+ * with one CTA per 16 state columns of each chain (about 2.5x slower per token
+ * at d = 112).  With chunk_len 16 or 32: an FFMA chunked kernel.  When
+ * state_in == state_out the launch is cooperative and every initial state is
+ * read before any final state is written.
  */
 int gdn_forward(const void* q, const void* k, const void* v,
                 const float* gate_logit, const float* beta_logit,
@@ -130,8 +147,9 @@ int gdn_forward_host(const void* h_q, const void* h_k, const void* h_v,
  * Workspace entry points.  The chunked method splits every chunk's work into a
  * state-independent half (gates, norms, the decayed key Gram matrix, the UT
  * inverse T = (I + A)^{-1} diag(beta), W = T diag(e^G) K and U = T V) and the
- * state chain.  gdn_forward runs the first half once per 16 state columns;
- * the *_ws calls run it once per chunk and head and hand the results to the
+ * state chain.  These calls keep every chain on its own group of CTAs (one
+ * per 16 state columns) over the whole sequence: they run the first half once
+ * per chunk and head and hand the results to the
  * CTAs of the head's state chain through a ring of records in `workspace`
  * (a few tens of MB, sized by gdn_workspace_bytes, reused chunk after chunk so
  * that it stays in L2).  Results equal gdn_forward's up to rounding.
@@ -313,8 +331,9 @@ int gdn_get_last_device_status(cudaStream_t stream);
  */
 int gdn_set_wait_limit_ns(unsigned long long ns);
 
-/* Which kernel the bf16 entry points dispatch to for the given sizes
- * (0 = FFMA chunked kernel, 1 = tensor-core chunked kernel). */
+/* Which kernel gdn_forward / gdn_state_step / gdn_forward_host dispatch to for
+ * the given sizes: 0 = FFMA chunked kernel, 1 = tensor-core kernel with one CTA
+ * per 16 state columns of each chain, 2 = sequence-parallel tensor-core kernel. */
 int gdn_bf16_path(int d_k, int d_v, int chunk_len);
 
 /* Library version, as major * 10000 + minor * 100 + patch. */

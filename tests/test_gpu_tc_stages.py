@@ -43,7 +43,8 @@ CASES = {
 
 
 def test_tensor_core_path_selected():
-    assert G.gdn_bf16_path(112, 112, 64) == 1
+    assert G.gdn_bf16_path(112, 112, 64) == 2      # the sequence-parallel kernel
+    assert G.gdn_bf16_path(128, 128, 64) == 1      # d = 128: the fused kernel
 
 
 @pytest.mark.parametrize("name", list(CASES))
