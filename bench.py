@@ -2,11 +2,18 @@
 """GDN forward benchmark on B200: tokens/s per layer on the minute-scale SANA-WM layer.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload minute|block|clip241|sessions]
 
-Workload: B = 1, H = 20, d_k = d_v = 112, T = 106,480 tokens (121 latent frames
-of 880 tokens), chunk 64, bf16 q/k/v/out, float32 logits and state, seeded
-synthetic inputs; one step = 20 layer calls back to back (one buffer set of
-1.9 GB, larger than the 126 MB L2, so no call finds its inputs in L2).
+Default workload (minute): B = 1, H = 20, d_k = d_v = 112, T = 106,480 tokens
+(121 latent frames of 880 tokens), chunk 64, bf16 q/k/v/out, float32 logits and
+state, seeded synthetic inputs; one step = 20 layer calls back to back (one
+buffer set of 1.9 GB, larger than the 126 MB L2, so no call finds its inputs in
+L2).  The other workloads: block (one 3-frame streaming block, T = 2,640, state
+in and out; 20 calls per step rotating over 8 buffer sets, 396 MB in all, so
+that no call finds its inputs in L2), clip241 (T = 27,280, zero initial state,
+20 layers per step) and sessions (4 independent sessions, 40 successive
+3-frame blocks per step through gdn_state_step with the state carried in
+place; every block its own inputs, 7.9 GB in all).
 
 Multi-GPU: one process per GPU (torchrun); the layer's (batch, head) chains are
 independent, so every rank runs the same per-GPU workload with no collective
@@ -36,7 +43,8 @@ METRIC = "GDN fwd tokens/s per layer (20 heads x d112) on 1 B200; % of roofline"
 UNIT = "tokens/s"
 BYTES_PER_TOKEN_HEAD = 900          # q, k, v in + out (bf16, d = 112) + beta logit (f32)
 CHUNKED_FLOPS_PER_TOKEN_HEAD = 146944   # 10 C d + 6 d^2 at C = 64, d = 112
-KERNEL_SOURCES = ["hybrid_linear_attention_frame_b200/csrc/gdn_ring.cu",
+KERNEL_SOURCES = ["hybrid_linear_attention_frame_b200/csrc/gdn_seq.cu",
+                  "hybrid_linear_attention_frame_b200/csrc/gdn_ring.cu",
                   "hybrid_linear_attention_frame_b200/csrc/gdn_tc.cu",
                   "hybrid_linear_attention_frame_b200/csrc/gdn_ffma.cu",
                   "hybrid_linear_attention_frame_b200/csrc/gdn_common.cuh",
@@ -59,9 +67,13 @@ def parse_args(argv=None):
     ap.add_argument("--gate-mode", choices=["token", "frame"], default="token",
                     help="token: a frame's gate at each of its tokens (gdn_forward*); frame: once, at "
                          "the frame's first token (gdn_forward_gated, gate_mode 1)")
-    ap.add_argument("--path", choices=["ws", "plain"], default="ws",
-                    help="ws: gdn_forward_ws (shared prep through a workspace ring); "
-                         "plain: gdn_forward (no workspace)")
+    ap.add_argument("--path", choices=["ws", "plain"], default="plain",
+                    help="plain: gdn_forward / gdn_state_step (sequence-parallel kernel, no workspace); "
+                         "ws: gdn_forward_ws / gdn_state_step_ws (shared prep through a workspace ring)")
+    ap.add_argument("--workload", choices=["minute", "block", "clip241", "sessions"], default="minute",
+                    help="minute: the minute-scale layer (default); block: one streaming block with state in "
+                         "and out; clip241: the 241-frame clip layer; sessions: 4 sessions x 40 blocks "
+                         "through gdn_state_step")
     ap.add_argument("--layer", choices=["gdn", "softmax"], default="gdn",
                     help="gdn: the GDN layer; softmax: the chunk-causal softmax attention layer "
                          "(gdn_softmax_attention, blocks of 3 frames, 2 cached blocks, 1 sink frame)")
@@ -283,7 +295,7 @@ def run_reference(args, w, rank, world):
     inp = make_inputs(w)
     threads = oracle_threads(w)
     budget = 150.0 / max(1, args.steps + args.warmup)      # whole run within a few minutes
-    layers = args.layers or w.layers
+    layers = calls_per_step(args, w)
     if args.layer == "softmax":
         per_call = min(args.cpu_seconds, budget)
         for _ in range(args.warmup):
@@ -303,9 +315,7 @@ def run_reference(args, w, rank, world):
         form = "forward plus backward token recurrence" if bidir else "token recurrence"
         sample = (f"float64 C {form}, first {n_tok} tokens of all {w.B * w.H} chains "
                   f"of one layer per step, {threads} OpenMP threads (host has {os.cpu_count()} cores)")
-        metric, config, cores = METRIC, workload_config(w, layers), threads
-        if bidir:
-            config["direction"] = "forward plus backward scan (gdn_forward_bidir)"
+        metric, config, cores = METRIC, run_config(args, w), threads
     return {"metric": metric, "value": value, "unit": UNIT, "impl": "reference",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -316,14 +326,66 @@ def run_reference(args, w, rank, world):
 
 
 def workload_config(w, layers):
-    return {"workload": f"{w.name}: minute-scale SANA-WM GDN layer, B={w.B} H={w.H} "
-                        f"T={w.T} d_k=d_v={w.d_k}, frame {w.frame_len} tokens, chunk {w.chunk_len}, "
-                        f"{layers} layers back-to-back per step",
+    what = {"minute": "minute-scale SANA-WM GDN layer", "block": "one SANA-WM streaming block (3 latent frames)",
+            "clip241": "241-frame clip GDN layer (31 latent frames)",
+            "sessions": "batched streaming sessions"}.get(w.name, w.name)
+    if w.name == "sessions":
+        per_step = (f"{w.blocks} successive blocks of {w.T} tokens per session per step, state carried "
+                    "block to block in place")
+        l2 = f"every block its own inputs ({w.blocks} sets, 7.9 GB)"
+        state = f"initial state N(0, {w.state_std}) per session (seed {w.session_seed_base} + s), carried"
+    elif w.name == "block":
+        per_step = f"{layers} calls per step over {BLOCK_SETS} buffer sets in rotation"
+        l2 = f"{BLOCK_SETS} rotating input sets, 396 MB in all vs the 126 MB L2"
+        state = f"state in N(0, {w.state_std}) and out"
+    else:
+        per_step = f"{layers} layers back-to-back per step"
+        l2 = "inputs larger than L2 ({:.2f} GB per layer vs 126 MB)".format(w.B * w.T * w.H * 900 / 1e9)
+        state = "zero initial state, final state written"
+    return {"workload": f"{w.name}: {what}, B={w.B} H={w.H} T={w.T} d_k=d_v={w.d_k}, frame {w.frame_len} "
+                        f"tokens, chunk {w.chunk_len}, {per_step}",
             "B": w.B, "H": w.H, "T": w.T, "d_k": w.d_k, "d_v": w.d_v, "frame_len": w.frame_len,
-            "chunk_len": w.chunk_len, "layers_per_step": layers,
-            "gate_logits": f"N({w.gate_mean}, {w.gate_std})", "seed": w.seed,
-            "l2": "inputs larger than L2 (1.9 GB per layer vs 126 MB)",
-            "parallelism": "weak: every rank runs the full layer set on its own GPU"}
+            "chunk_len": w.chunk_len, "calls_per_step": layers,
+            "gate_logits": f"N({w.gate_mean}, {w.gate_std})", "seed": w.seed, "state": state,
+            "l2": l2, "parallelism": "weak: every rank runs the full workload on its own GPU"}
+
+
+BLOCK_SETS = 8
+
+
+def workload_of(args):
+    from workloads import BLOCK, CLIP241, MINUTE, SESSIONS
+    return {"minute": MINUTE, "block": BLOCK, "clip241": CLIP241, "sessions": SESSIONS}[args.workload]
+
+
+def calls_per_step(args, w):
+    if w.name == "sessions":
+        return w.blocks
+    return args.layers or 20
+
+
+def run_config(args, w):
+    """The config object of the JSON line; the same for both arms of one invocation."""
+    layers = calls_per_step(args, w)
+    bidir = args.direction == "bidir"
+    gate_mode = args.gate_mode == "frame"
+    stream_step = w.name == "sessions"
+    if bidir:
+        api = "gdn_forward_bidir (C ABI, device buffers, caller workspace reused by every layer)"
+    elif gate_mode:
+        api = "gdn_forward_gated" + (" with a workspace" if args.path == "ws" else "") + " (C ABI, device buffers)"
+    elif stream_step:
+        api = ("gdn_state_step_ws (C ABI, device buffers, caller workspace)" if args.path == "ws"
+               else "gdn_state_step (C ABI, device buffers, state in place)")
+    else:
+        api = ("gdn_forward_ws (C ABI, device buffers, caller workspace reused by every layer)"
+               if args.path == "ws" else "gdn_forward (C ABI, device buffers, no workspace)")
+    cfg = dict(workload_config(w, layers),
+               direction=("forward plus backward scan (gdn_forward_bidir)" if bidir else "forward scan"),
+               gate_placement=("once per frame, at its first token (gate_mode 1)" if gate_mode
+                               else "at every token of the frame"),
+               api=api)
+    return cfg
 
 
 # ----------------------------------------------------------------------------
@@ -474,65 +536,101 @@ def run_softmax(args, w, rank, world, local):
 # our arm
 # ----------------------------------------------------------------------------
 
-def run_ours(args, w, rank, world, local):
+def upload_sets(w, device):
+    """Host (pinned later for e2e) and device copies of the workload's input sets.
+
+    Returns a list of dicts with host tensors h_q, h_k, h_v, h_g, h_b, h_s (state or
+    None) and their device copies q, k, v, g, b, s."""
     import numpy as np
     import torch
+    from workloads import bf16_bits, make_inputs, make_session_blocks
+
+    def bf16(x):
+        return torch.from_numpy(bf16_bits(x).view(np.int16)).view(torch.bfloat16)
+
+    if w.name == "sessions":
+        state0, blocks = make_session_blocks(w)
+        inps = blocks
+        states = [state0] + [None] * (len(blocks) - 1)
+    else:
+        n = BLOCK_SETS if w.name == "block" else 1
+        inps = [make_inputs(w, seed=w.seed + i) for i in range(n)]
+        states = [x.state for x in inps]
+    sets = []
+    for inp, st in zip(inps, states):
+        h = {"h_q": bf16(inp.q), "h_k": bf16(inp.k), "h_v": bf16(inp.v),
+             "h_g": torch.from_numpy(np.ascontiguousarray(inp.gate)),
+             "h_b": torch.from_numpy(np.ascontiguousarray(inp.beta)),
+             "h_s": None if st is None else torch.from_numpy(np.ascontiguousarray(st, dtype=np.float32))}
+        for key in ("q", "k", "v", "g", "b", "s"):
+            h[key] = None if h["h_" + key] is None else h["h_" + key].to(device)
+        sets.append(h)
+    return sets, inps[0]
+
+
+def run_ours(args, w, rank, world, local):
+    import torch
     import hybrid_linear_attention_frame_b200 as G
-    from workloads import bf16_bits, make_inputs
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     dist_init("nccl", world)
-    layers = args.layers or w.layers
-    G.load()
-
-    inp = make_inputs(w)
-    def bf16(x):
-        return torch.from_numpy(bf16_bits(x).view(np.int16)).view(torch.bfloat16)
-    h_q, h_k, h_v = bf16(inp.q), bf16(inp.k), bf16(inp.v)
-    h_g = torch.from_numpy(inp.gate)
-    h_b = torch.from_numpy(inp.beta)
-    q, k, v, g, b = (x.to(device) for x in (h_q, h_k, h_v, h_g, h_b))
-    out = torch.empty_like(v)
+    layers = calls_per_step(args, w)
+    lib = G.load()
+    sets, inp0 = upload_sets(w, device)
+    stream_step = w.name == "sessions"
+    out = torch.empty_like(sets[0]["v"])
     st_out = torch.empty((w.B, w.H, w.d_k, w.d_v), dtype=torch.float32, device=device)
+    if stream_step:
+        st_out.copy_(sets[0]["s"])             # the sessions' state, carried in place
     stream = torch.cuda.current_stream(device)
     sptr = stream.cuda_stream
-    lib = G.load()
     dims = (w.B, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.chunk_len)
-    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), b.data_ptr(), None,
-            st_out.data_ptr(), out.data_ptr())
     bidir = args.direction == "bidir"
-    if bidir and (args.gate_mode == "frame" or args.path == "plain"):
-        raise SystemExit("--direction bidir takes the gate at every token and its own workspace")
+    gate_mode = 1 if args.gate_mode == "frame" else 0
+    if bidir and (gate_mode or args.path == "plain" or w.name != "minute"):
+        raise SystemExit("--direction bidir: minute workload, gate at every token, --path ws")
+    if gate_mode and stream_step:
+        raise SystemExit("--gate-mode frame applies to the layer workloads")
     use_ws = args.path == "ws" and G.gdn_workspace_bytes(*dims[:5], w.chunk_len) > 0
     if bidir:
         ws = G.bidir_workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.chunk_len, device)
     else:
         ws = G.workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.chunk_len, device) if use_ws else None
     ws_args = (ws.data_ptr(), ws.numel()) if ws is not None else (None, 0)
+    with_state_in = w.name == "block" or stream_step
 
-    gate_mode = 1 if args.gate_mode == "frame" else 0
-
-    def layer_call():
+    def layer_call(i):
+        x = sets[i % len(sets)]
+        ptr = (x["q"].data_ptr(), x["k"].data_ptr(), x["v"].data_ptr(), x["g"].data_ptr(), x["b"].data_ptr())
         if bidir:
-            st = lib.gdn_forward_bidir(q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), b.data_ptr(),
-                                       out.data_ptr(), *dims, *ws_args, sptr)
-            if st != 0:
-                raise G.GdnError(st, "gdn_forward_bidir")
-            return
-        if gate_mode:
-            st = lib.gdn_forward_gated(*ptrs, *dims, gate_mode, *ws_args, sptr)
-        elif use_ws:
-            st = lib.gdn_forward_ws(*ptrs, *dims, *ws_args, sptr)
+            st = lib.gdn_forward_bidir(*ptr, out.data_ptr(), *dims, *ws_args, sptr)
+            name = "gdn_forward_bidir"
+        elif stream_step:
+            if use_ws:
+                st = lib.gdn_state_step_ws(*ptr, st_out.data_ptr(), out.data_ptr(), *dims, *ws_args, sptr)
+                name = "gdn_state_step_ws"
+            else:
+                st = lib.gdn_state_step(*ptr, st_out.data_ptr(), out.data_ptr(), *dims, sptr)
+                name = "gdn_state_step"
         else:
-            st = lib.gdn_forward(*ptrs, *dims, sptr)
+            s_in = x["s"].data_ptr() if (with_state_in and x["s"] is not None) else None
+            args_ = (*ptr, s_in, st_out.data_ptr(), out.data_ptr())
+            if gate_mode:
+                st = lib.gdn_forward_gated(*args_, *dims, gate_mode, *ws_args, sptr)
+                name = "gdn_forward_gated"
+            elif use_ws:
+                st = lib.gdn_forward_ws(*args_, *dims, *ws_args, sptr)
+                name = "gdn_forward_ws"
+            else:
+                st = lib.gdn_forward(*args_, *dims, sptr)
+                name = "gdn_forward"
         if st != 0:
-            raise G.GdnError(st, "gdn_forward_gated" if gate_mode else
-                             ("gdn_forward_ws" if use_ws else "gdn_forward"))
+            raise G.GdnError(st, name)
 
     for _ in range(args.warmup):
-        for _ in range(layers):
-            layer_call()
+        for i in range(layers):
+            layer_call(i)
     torch.cuda.synchronize(device)
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -547,13 +645,13 @@ def run_ours(args, w, rank, world, local):
     barrier(world, device)
     torch.cuda.synchronize(device)
     t_start.record(stream)
-    i = 0
+    n = 0
     for _ in range(args.steps):
-        for _ in range(layers):
-            ev[i][0].record(stream)
-            layer_call()
-            ev[i][1].record(stream)
-            i += 1
+        for i in range(layers):
+            ev[n][0].record(stream)
+            layer_call(i)
+            ev[n][1].record(stream)
+            n += 1
     t_end.record(stream)
     torch.cuda.synchronize(device)
     barrier(world, device)
@@ -566,64 +664,49 @@ def run_ours(args, w, rank, world, local):
     tokens_per_rank = w.B * w.T * layers * args.steps
     value, slowest = aggregate_throughput(tokens_per_rank, elapsed_s, world, device)
     ms_per_step = slowest * 1e3 / args.steps
-    launch_ms = [s.elapsed_time(e) for (s, e) in ev]
+    launch_ms = [a_.elapsed_time(b_) for (a_, b_) in ev]
     avg_launch_s = statistics.mean(launch_ms) / 1e3
 
     peaks, peak_kind = measured_peaks()
-    abytes = algorithmic_bytes(w, state_in=False, state_out=not bidir)
+    abytes = algorithmic_bytes(w, state_in=with_state_in, state_out=not bidir)
     achieved = abytes / avg_launch_s / 1e9
     traffic, traffic_kernel = recorded_traffic()
-    path = G.gdn_bf16_path(w.d_k, w.d_v, w.chunk_len)
     if bidir:
         kernel = "gdn_forward_bidir (one layer call: reverse copy, 2 x gdn_ring_kernel, combine)"
     elif use_ws:
         kernel = "gdn_ring_kernel"
+    elif G.gdn_bf16_path(w.d_k, w.d_v, w.chunk_len) == 2:
+        kernel = "gdn_seq_kernel"
     else:
-        kernel = "gdn_chunk_tc_kernel" if path == 1 else "chunk_ffma_kernel<bf16,64>"
+        kernel = "gdn_chunk_tc_kernel" if G.gdn_bf16_path(w.d_k, w.d_v, w.chunk_len) == 1 \
+            else "chunk_ffma_kernel<bf16,64>"
+    flops_scans = 2 if bidir else 1
+    flops = flops_scans * CHUNKED_FLOPS_PER_TOKEN_HEAD * w.B * w.T * w.H
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic if traffic_kernel == kernel else None,
+                "traffic": traffic if (traffic_kernel == kernel and w.name == "minute") else None,
                 "kernel": kernel, "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
                 "algorithmic_bytes_per_launch": abytes,
                 "avg_launch_us": round(avg_launch_s * 1e6, 2),
-                "tensor_flops_frac": round(
-                    CHUNKED_FLOPS_PER_TOKEN_HEAD * w.B * w.T * w.H / avg_launch_s / 1e12
-                    / peaks["bf16_tflops"], 4),
+                "tensor_flops_frac": round(flops / avg_launch_s / 1e12 / peaks["bf16_tflops"], 4),
                 "roofline_frac": round(max(abytes / (peaks["hbm_gbs"] * 1e9),
-                                           CHUNKED_FLOPS_PER_TOKEN_HEAD * w.B * w.T * w.H
-                                           / (peaks["bf16_tflops"] * 1e12)) / avg_launch_s, 4)}
-
-    flops_scans = 2 if bidir else 1
-    roofline["tensor_flops_frac"] = round(roofline["tensor_flops_frac"] * flops_scans, 4)
-    roofline["roofline_frac"] = round(max(abytes / (peaks["hbm_gbs"] * 1e9),
-                                          flops_scans * CHUNKED_FLOPS_PER_TOKEN_HEAD * w.B * w.T * w.H
-                                          / (peaks["bf16_tflops"] * 1e12)) / avg_launch_s, 4)
+                                           flops / (peaks["bf16_tflops"] * 1e12)) / avg_launch_s, 4)}
+    if stream_step:
+        roofline["per_block_us"] = round(avg_launch_s * 1e6, 2)
 
     e2e = None
     if not args.no_e2e and not bidir:
-        e2e = run_e2e(lib, G, w, device, stream, (h_q, h_k, h_v, h_g, h_b),
-                      (q, k, v, g, b), out, st_out, world, max(2, min(args.steps, 3)), ws)
+        e2e = run_e2e(lib, G, w, device, stream, sets, out, st_out, world,
+                      max(2, min(args.steps, 3)) if not stream_step else 1, layers if stream_step else 1, ws)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, inp, args.cpu_seconds, bidir=bidir)
+        cpu = cpu_baseline(w, inp0, args.cpu_seconds, bidir=bidir)
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": dict(workload_config(w, layers),
-                           direction=("forward plus backward scan (gdn_forward_bidir)" if bidir
-                                      else "forward scan"),
-                           gate_placement=("once per frame, at its first token (gate_mode 1)" if gate_mode
-                                           else "at every token of the frame"),
-                           api=("gdn_forward_bidir (C ABI, device buffers, workspace "
-                                f"{ws.numel() / 2**20:.1f} MiB reused by every layer)") if bidir
-                           else (("gdn_forward_gated" if gate_mode else "gdn_forward_ws") +
-                                 " (C ABI, device buffers, workspace "
-                                 f"{ws.numel() / 2**20:.1f} MiB reused by every layer)") if use_ws
-                           else ("gdn_forward_gated" if gate_mode else "gdn_forward") +
-                           " (C ABI, device buffers)"),
+            "data": "synthetic", "config": run_config(args, w),
             "roofline": roofline,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * layers * (4 if bidir else 1),
             "clocks": clock_rec}
@@ -634,45 +717,58 @@ def run_ours(args, w, rank, world, local):
     return line if rank == 0 else None
 
 
-def run_e2e(lib, G, w, device, stream, host_src, dev, out, st_out, world, steps, ws=None):
+def run_e2e(lib, G, w, device, stream, sets, out, st_out, world, steps, calls, ws=None):
     """The same metric through gdn_forward_host(_ws): pinned host inputs copied
-    in, output and final state copied out, every step."""
+    in, output and final state copied out, every call (a layer, or a streaming
+    block whose state goes in and out through the host)."""
     import torch
-    hq, hk, hv, hg, hb = (x.pin_memory() for x in host_src)
+    pinned = []
+    for x in sets[:max(1, min(len(sets), calls))]:
+        pinned.append({key: (None if x["h_" + key] is None else x["h_" + key].pin_memory())
+                       for key in ("q", "k", "v", "g", "b", "s")})
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h_st = torch.empty(st_out.shape, dtype=torch.float32).pin_memory()
-    q, k, v, g, b = dev
+    x0 = sets[0]
     sptr = stream.cuda_stream
-
-    host_args = (hq.data_ptr(), hk.data_ptr(), hv.data_ptr(), hg.data_ptr(), hb.data_ptr(), None,
-                 h_st.data_ptr(), h_out.data_ptr(), q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                 g.data_ptr(), b.data_ptr(), st_out.data_ptr(), out.data_ptr(),
-                 w.B, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.chunk_len)
     api = "gdn_forward_host_ws" if ws is not None else "gdn_forward_host"
+    stream_step = w.name == "sessions"
 
-    def call():
-        if ws is not None:
-            st = lib.gdn_forward_host_ws(*host_args, ws.data_ptr(), ws.numel(), sptr)
+    def call(i):
+        hp = pinned[i % len(pinned)]
+        if stream_step:
+            h_s = h_st if i > 0 else hp["s"]        # the state goes out to the host and back in
         else:
-            st = lib.gdn_forward_host(*host_args, sptr)
+            h_s = hp["s"]
+        a = (hp["q"].data_ptr(), hp["k"].data_ptr(), hp["v"].data_ptr(), hp["g"].data_ptr(), hp["b"].data_ptr(),
+             None if h_s is None else h_s.data_ptr(), h_st.data_ptr(), h_out.data_ptr(),
+             x0["q"].data_ptr(), x0["k"].data_ptr(), x0["v"].data_ptr(), x0["g"].data_ptr(), x0["b"].data_ptr(),
+             st_out.data_ptr(), out.data_ptr(), w.B, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.chunk_len)
+        if ws is not None:
+            st = lib.gdn_forward_host_ws(*a, ws.data_ptr(), ws.numel(), sptr)
+        else:
+            st = lib.gdn_forward_host(*a, sptr)
         if st != 0:
             raise G.GdnError(st, api)
 
-    call()
+    call(0)
     barrier(world, device)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(steps):
-        call()
+        for i in range(calls):
+            call(i)
     t1.record(stream)
     torch.cuda.synchronize(device)
     elapsed = t0.elapsed_time(t1) / 1e3
-    value, _ = aggregate_throughput(w.B * w.T * steps, elapsed, world, device)
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg, hb))
+    value, _ = aggregate_throughput(w.B * w.T * steps * calls, elapsed, world, device)
+    hp = pinned[0]
+    h2d = sum(hp[key].numel() * hp[key].element_size() for key in ("q", "k", "v", "g", "b"))
+    if hp["s"] is not None or stream_step:
+        h2d += h_st.numel() * 4
     d2h = h_out.numel() * h_out.element_size() + h_st.numel() * 4
-    return {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps,
-            "api": f"{api} (C ABI, pinned host buffers, one layer per step)"}
+    return {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d * calls,
+            "d2h_bytes_per_step": d2h * calls, "steps": steps,
+            "api": f"{api} (C ABI, pinned host buffers, {calls} call(s) per step)"}
 
 
 def run_profile_case(w, tokens, path="ws"):
@@ -729,8 +825,9 @@ def run_profile_case_softmax(w, tokens):
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_env()
-    from workloads import MINUTE
-    w = MINUTE
+    w = workload_of(args)
+    if args.layer == "softmax" and w.name != "minute":
+        raise SystemExit("--layer softmax runs on the minute workload")
     if args.profile_tokens > 0 and args.layer == "softmax":
         return run_profile_case_softmax(w, args.profile_tokens)
     if args.profile_tokens > 0:

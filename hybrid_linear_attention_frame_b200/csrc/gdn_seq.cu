@@ -31,9 +31,10 @@
 // state is read back, the next chunk's decay e^{G_L} is applied to it, so that
 // MMA2 adds onto the already decayed state.
 //
-// Warp roles (16 warps): 0 loads q and k tiles (TMA), 1 issues the Gram MMAs,
+// Warp roles (20 warps): 0 loads q and k tiles (TMA), 1 issues the Gram MMAs,
 // 2 issues the chain MMAs, 3 issues the W/U MMAs and loads v tiles, 4-11 prep,
-// 12-15 chain and output.  Hand-offs are mbarriers; every wait is bounded and
+// 12-19 chain and output (two warps per TMEM lane quarter, each on half of the
+// d_v columns).  Hand-offs are mbarriers; every wait is bounded and
 // gives up with GDN_ERR_TIMEOUT.
 #include <cooperative_groups.h>
 #include <cudaTypedefs.h>
@@ -49,12 +50,14 @@ using namespace sm100;
 using tc::kC;
 using tc::kXS;
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 640;
 constexpr int kMaxAtoms = 7;                 // d_k, d_v <= 112 (16-column atoms)
 constexpr int kWarpLoadKQ = 0, kWarpGram = 1, kWarpChainMma = 2, kWarpWU = 3;
 constexpr int kPrepWarp0 = 4, kChainWarp0 = 12;
 constexpr int kPrepThreads = 256;
 constexpr uint32_t kBarPrep = 1;             // named barrier of the prep warps (3: the UT inverse's)
+constexpr uint32_t kBarOut = 2;              // named barrier of the four output warps
+constexpr uint32_t kBarA = 4;                // the four prep warps that form A and invert I + A
 
 // product of gates over a warm-up stretch below which the state entering it is dropped: 2^-48
 constexpr float kWarmupLogDecay = 48.0f * 0.693147181f;
@@ -72,7 +75,7 @@ constexpr uint32_t kColSacc = 384;           // state: d_k lanes x d_v columns
 constexpr uint32_t kAtomKQW = 6144;          // per d_k atom: K rows | Q rows | W rows (64 each)
 constexpr uint32_t kAtQ = 2048, kAtW = 4096;
 constexpr uint32_t kStageSc = kMaxAtoms * kAtomKQW;          // chain scalars of the stage
-constexpr uint32_t kStageBytes = kStageSc + 1024;
+constexpr uint32_t kStageBytes = kStageSc + 2048;
 constexpr uint32_t kOffV = 2 * kStageBytes;                  // v tile, d_v atoms of 64 rows
 constexpr uint32_t kAtomV = 2048;
 constexpr uint32_t kTile = 8192;                             // 64 x 64 bf16, 128-byte swizzle
@@ -84,13 +87,13 @@ constexpr uint32_t kOffS = kOffT + kTile;                    // S bf16, d_v atom
 constexpr uint32_t kAtomS = 112 * 32;
 constexpr uint32_t kOffEp = kOffS + kMaxAtoms * kAtomS;      // E' bf16, d_v atoms of 64 rows
 constexpr uint32_t kAtomE = 64 * 32;
-constexpr uint32_t kOffE = kOffEp + kMaxAtoms * kAtomE;      // E bf16
+constexpr uint32_t kOffE = kOffEp + kMaxAtoms * kAtomE;      // E bf16; then the output rows [64][d_v] bf16
 constexpr uint32_t kOffAXI = kOffE + kMaxAtoms * kAtomE;     // fp32 [64][kXS]: A / (I+A)^{-1}
 constexpr uint32_t kScFloats = 13 * 64 + 16;
 constexpr uint32_t kOffSc = kOffAXI + 64 * kXS * 4;          // prep scalar table
 constexpr uint32_t kOffBar = kOffSc + kScFloats * 4;
 enum : uint32_t {
-    B_FULL = 0,       // [2] q/k tiles of a stage landed
+    B_FULL = 0,       // [2] q/k tiles of a stage landed and its gates written
     B_SFREE = 2,      // [2] chain MMAs done with a stage (and with its P)
     B_VFULL = 4,      // v tile landed
     B_VFREE = 5,      // U MMA done with the v tile
@@ -106,7 +109,8 @@ enum : uint32_t {
     B_PEGO = 17,      // E written and Q S scaled
     B_M2 = 18,        // MMA2 done
     B_PEDONE = 19,    // P E done
-    kNumBars = 20,
+    B_OFREE = 20,     // output staging (the E tile) read by its TMA store
+    kNumBars = 21,
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
@@ -127,8 +131,10 @@ enum : uint32_t {
     SC_BGK = 704,    // beta_j e^{G_j} / |k_j|
     SC_MISC = 768,
 };
-// chain scalars of a stage (floats): e^G/|q| and e^{G_L-G}/|k| (0 beyond the chunk)
-enum : uint32_t { CS_GQ = 0, CS_DL = 64 };
+// per-chunk scalars in a stage (floats).  Written by the q/k loader warp: the
+// cumulative log-gate G_i, beta_i (both 0 past the chunk's valid length) and the
+// chunk's decay e^{G_L}.  Written by the prep: e^G/|q| and e^{G_L-G}/|k|.
+enum : uint32_t { CS_GQ = 0, CS_DL = 64, CS_G = 128, CS_BETA = 192, CS_GL = 256 };
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffP % 1024 == 0 && kOffTp % 1024 == 0 && kStageBytes % 1024 == 0, "SW128 alignment");
@@ -141,7 +147,7 @@ static_assert(kOffAXI % 16 == 0 && kOffSc % 16 == 0 && kOffBar % 8 == 0, "alignm
 constexpr uint32_t kIdGram = idesc_bf16(128, 128, false, false);
 
 __host__ __device__ constexpr uint32_t bar_count(uint32_t i) {
-    return (i == B_SREADY || i == B_PEGO) ? 4u : (i == B_EQFREE || i == B_EQFREE + 1 || i == B_EREADY) ? 2u : 1u;
+    return (i == B_SREADY || i == B_PEGO) ? 8u : (i == B_EREADY) ? 4u : (i == B_FULL || i == B_FULL + 1) ? 2u : 1u;
 }
 
 // descriptors: K-major / MN-major 32-byte swizzle (8-row groups 256 B apart), K-major 128-byte swizzle
@@ -175,7 +181,33 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
                  : "memory");
 }
 
+// Arrive without release semantics: for hand-offs that order nothing but TMEM
+// reads already completed (tcgen05.wait::ld), so that the arrive does not wait
+// for this thread's global stores in flight.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.relaxed.cta.shared::cta.b64 st, [%0];\n\t}"
+                 :: "r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Read 16-column pieces [0, n) of this warp's 32 TMEM lanes starting at `taddr`,
+// kBatch pieces per wait (so that the load latency is paid once per batch), and
+// hand each piece to f(piece, values).  Warp-collective: n must be warp-uniform.
+template <int kBatch = 2, typename F>
+__device__ __forceinline__ void tmem_pieces(uint32_t taddr, int n, F&& f) {
+#pragma unroll 1
+    for (int a0 = 0; a0 < n; a0 += kBatch) {
+        float v[kBatch][16];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j)
+            if (a0 + j < n) tmem_ld16(taddr + 16u * (uint32_t)(a0 + j), v[j]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j)
+            if (a0 + j < n) f(a0 + j, v[j]);
+    }
+}
 
 __device__ __forceinline__ float softplus_fast(float x) { return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x))); }
 __device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
@@ -290,7 +322,7 @@ __device__ __forceinline__ float chunk_decay(const FwdParams& p, int b, int h, i
 
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const SeqArgs a)
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const SeqArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -315,6 +347,7 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
+        if (a.p.out) tma_prefetch_desc(&tm_o);
     }
     if (warp == kWarpWU) {
         // warm-up start of the first piece (see the file comment)
@@ -344,13 +377,17 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     // Chain warps: S tile and SACC for the first chunk of a piece (state_in or zero),
     // then SREADY.  SACC holds e^{G_L} S for the chunk about to run.
+    // chain warp: TMEM lane quarter q, and the half [a_lo, a_lo + na) of the d_v atoms
+    const int cq = warp & 3, chf = (warp - kChainWarp0) >> 2;
+    const int c_alo = chf ? (nav + 1) / 2 : 0, c_na = chf ? nav - (nav + 1) / 2 : (nav + 1) / 2;
     auto chain_init = [&](const Piece& pc) {
-        const int q = warp - kChainWarp0, row = 32 * q + lane;
+        const int q = cq, row = 32 * q + lane;
+        // (read from the gate logits directly: the first piece is set up before the loaders start)
         const float gl = __expf(-chunk_decay(p, pc.b, pc.h, pc.cw, lane));
         const float* si = (pc.rd && row < dk)
                               ? p.state_in + (((size_t)pc.b * p.H + pc.h) * dk + row) * (size_t)dv
                               : nullptr;
-        for (int at = 0; at < nav; ++at) {
+        for (int at = c_alo; at < c_alo + c_na; ++at) {
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.0f;
@@ -389,6 +426,19 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         int issued = 0;
         for (Cursor cu(a, P, warm0); cu.valid(); cu.next()) {
             const int n = cu.n, s = n & 1;
+            // the chunk's gate and beta logits: the only global loads of a chunk besides the
+            // tiles, made by this warp (so that no compute warp waits for them at a barrier)
+            // and issued before the wait for the stage, which hides their latency
+            const int L = cu.L(), i0 = 2 * lane, t0 = cu.c * kC + i0;
+            float g0 = 0.f, g1 = 0.f, r0 = 0.f, r1 = 0.f;
+            if (i0 < L) {
+                g0 = __ldg(p.gate + ((size_t)cu.pc.b * p.F + t0 / p.frame_len) * p.H + cu.pc.h);
+                r0 = __ldg(p.beta + ((size_t)cu.pc.b * p.T + t0) * p.H + cu.pc.h);
+            }
+            if (i0 + 1 < L) {
+                g1 = __ldg(p.gate + ((size_t)cu.pc.b * p.F + (t0 + 1) / p.frame_len) * p.H + cu.pc.h);
+                r1 = __ldg(p.beta + ((size_t)cu.pc.b * p.T + t0 + 1) * p.H + cu.pc.h);
+            }
             if (n >= 2) {
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFREE + s), (uint32_t)(((n - 2) >> 1) & 1),
                                                        abort_flag, lim, 21));
@@ -403,7 +453,25 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 cu.pc.b);
                 }
             }
-            __syncwarp();
+            // G (warp scan of the log-gates), beta and e^{G_L} into the stage
+            {
+                float* cs = reinterpret_cast<float*>(gb + (uint32_t)s * kStageBytes + kStageSc);
+                const float la0 = (i0 < L && gate_applies(p, t0)) ? -softplus_fast(g0) : 0.0f;
+                const float la1 = (i0 + 1 < L && gate_applies(p, t0 + 1)) ? -softplus_fast(g1) : 0.0f;
+                float x = la0 + la1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                cs[CS_G + i0] = x - la1;
+                cs[CS_G + i0 + 1] = x;
+                cs[CS_BETA + i0] = (i0 < L) ? sigmoid_fast(r0) : 0.0f;
+                cs[CS_BETA + i0 + 1] = (i0 + 1 < L) ? sigmoid_fast(r1) : 0.0f;
+                if (lane == 31) cs[CS_GL] = __expf(x);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_FULL + s));
+            }
             issued = n + 1;
         }
         if (!ok && lane == 0)
@@ -532,62 +600,33 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float* MSf = reinterpret_cast<float*>(gb + kOffT);
         const uint32_t tg = tmem + kColG;
         bool ok = true;
-        // gate and beta logits of the next chunk, loaded one chunk ahead (warp pw 0)
-        float pg0 = 0.f, pg1 = 0.f, pb0 = 0.f, pb1 = 0.f;
-        auto load_logits = [&](const Cursor& c) {
-            const int L = c.L(), i0 = 2 * lane, t0 = c.c * kC + i0;
-            pg0 = pg1 = pb0 = pb1 = 0.0f;
-            if (i0 < L) {
-                pg0 = __ldg(p.gate + ((size_t)c.pc.b * p.F + t0 / p.frame_len) * p.H + c.pc.h);
-                pb0 = __ldg(p.beta + ((size_t)c.pc.b * p.T + t0) * p.H + c.pc.h);
-            }
-            if (i0 + 1 < L) {
-                pg1 = __ldg(p.gate + ((size_t)c.pc.b * p.F + (t0 + 1) / p.frame_len) * p.H + c.pc.h);
-                pb1 = __ldg(p.beta + ((size_t)c.pc.b * p.T + t0 + 1) * p.H + c.pc.h);
-            }
-        };
-        Cursor cn(a, P, warm0);
-        if (pw == 0 && cn.valid()) load_logits(cn);
-        for (Cursor cu(a, P, warm0); cu.valid(); cu.next()) {
+        // Per chunk: front (the stage's gates, norms, A and P from the Gram), the UT
+        // inverse and T, T', then back (-W beside Q once the U and W MMAs are done).
+        auto front = [&](const Cursor& cu) -> bool {
             const int n = cu.n, s = n & 1, L = cu.L();
             float* cs = reinterpret_cast<float*>(gb + (uint32_t)s * kStageBytes + kStageSc);
-            const uint32_t stg = base + (uint32_t)s * kStageBytes;
-            // ---- gates: G (warp scan), beta; then the decay tables ----
-            if (pw == 0) {
-                const int i0 = 2 * lane, t0 = cu.c * kC + i0;
-                const float la0 = (i0 < L && gate_applies(p, t0)) ? -softplus_fast(pg0) : 0.0f;
-                const float la1 = (i0 + 1 < L && gate_applies(p, t0 + 1)) ? -softplus_fast(pg1) : 0.0f;
-                float x = la0 + la1;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, off);
-                    if (lane >= off) x += y;
-                }
-                sc[SC_G + i0] = x - la1;
-                sc[SC_G + i0 + 1] = x;
-                sc[SC_BETA + i0] = (i0 < L) ? sigmoid_fast(pb0) : 0.0f;
-                sc[SC_BETA + i0 + 1] = (i0 + 1 < L) ? sigmoid_fast(pb1) : 0.0f;
-                cn.next();
-                if (cn.valid()) load_logits(cn);
-            }
-            named_bar_sync(kBarPrep, kPrepThreads);
+            // ---- the stage's gates written, the Gram done ----
+            ok = mbar_wait(bar(B_FULL + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 43);
+            ok = ok && mbar_wait(bar(B_G1), (uint32_t)(n & 1), abort_flag, lim, 41);
+            if (!group_all(kBarPrep, kPrepThreads, ok)) return false;
+            // ---- G and beta from the stage; the decay tables ----
             {
-                const float GL = sc[SC_G + 63];
+                const float GL = cs[CS_G + 63];
                 const int idx = pt;
                 if (idx < 64) {
                     const int i = idx;
-                    const float Gi = sc[SC_G + i];
+                    const float Gi = cs[CS_G + i];
+                    sc[SC_G + i] = Gi;
+                    sc[SC_BETA + i] = cs[CS_BETA + i];
                     sc[SC_GAM + i] = __expf(Gi);
                     sc[SC_DL + i] = (i < L) ? __expf(GL - Gi) : 0.0f;
-                    sc[SC_EXR + i] = (i >= 16) ? __expf(Gi - sc[SC_G + 16 * (i >> 4) - 1]) : 1.0f;
+                    sc[SC_EXR + i] = (i >= 16) ? __expf(Gi - cs[CS_G + 16 * (i >> 4) - 1]) : 1.0f;
                 } else {
                     const int bi = 1 + (idx - 64) / 64, j = idx & 63;
-                    sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? __expf(sc[SC_G + 16 * bi - 1] - sc[SC_G + j]) : 0.0f;
+                    sc[SC_EXC + 64 * bi + j] = (j < 16 * bi) ? __expf(cs[CS_G + 16 * bi - 1] - cs[CS_G + j]) : 0.0f;
                 }
             }
-            // ---- Gram done (this vote is also the barrier after the tables) ----
-            ok = mbar_wait(bar(B_G1), (uint32_t)(n & 1), abort_flag, lim, 41);
-            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            named_bar_sync(kBarPrep, kPrepThreads);
             tc_fence_after();
             // ---- norms from the Gram diagonal: |k_i|^2 (lanes 0-63), |q_i|^2 (lanes 64-127) ----
             if (pw < 4) {
@@ -612,7 +651,11 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
             named_bar_sync(kBarPrep, kPrepThreads);
-            // ---- A (fp32, transposed above the diagonal of AXI) and P (bf16 tile P[s]) ----
+            return true;
+        };
+        // A (fp32, transposed above the diagonal of AXI; TMEM lanes 0-63) and P (bf16
+        // tile P[s]; lanes 64-127) from the Gram, row 32 (qtr & 1) + lane of each warp.
+        auto gram_epilogue = [&](int s) {
             {
                 const uint32_t ptile = base + kOffP + kTile * (uint32_t)s;
                 const int ch = pw >> 2;
@@ -661,12 +704,18 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     }
                 }
             }
+        };
+        // The warps on TMEM lanes 0-63 (qtr 0, 1) form A and then invert I + A; the
+        // warps on lanes 64-127 form P meanwhile (P is needed only by the chain).
+        auto inverse_t = [&](int s) {
+            gram_epilogue(s);
+            if (qtr < 2) {
+                named_bar_sync(kBarA, 128);      // A complete
+                tc::unit_lower_inverse_64(AXI, MSf, 32 * ((pw & 1) | ((pw >> 2) << 1)) + lane);
+            }
             tc_fence_before();
             named_bar_sync(kBarPrep, kPrepThreads);
             if (pt == 0) mbar_arrive(bar(B_GFREE));       // the Gram accumulator may be overwritten
-            // ---- (I + A)^{-1} (warps 4-7) ----
-            if (pw < 4) tc::unit_lower_inverse_64(AXI, MSf, pt);
-            named_bar_sync(kBarPrep, kPrepThreads);
             // ---- T = (I+A)^{-1} diag(beta), T' = T diag(beta e^G / |k|): bf16 tiles ----
             {
                 const int i = pt >> 2, jb = 16 * (pt & 3);
@@ -694,18 +743,20 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             fence_proxy_async_smem();
             named_bar_sync(kBarPrep, kPrepThreads);
             if (pt == 0) mbar_arrive(bar(B_TREADY));
+        };
+        auto back = [&](int n) -> bool {
+            const int s = n & 1;
+            const uint32_t stg = base + (uint32_t)s * kStageBytes;
             // ---- U and W done: -W beside Q, then clear lanes 0-63 of EQS ----
             ok = mbar_wait(bar(B_WU), (uint32_t)(n & 1), abort_flag, lim, 42);
-            if (!group_all(kBarPrep, kPrepThreads, ok)) { ok = false; break; }
+            if (!group_all(kBarPrep, kPrepThreads, ok)) return false;
             tc_fence_after();
             if (qtr < 2) {
                 const int i = 32 * qtr + lane;
                 const uint32_t eq = tlane(tmem + kColEQS + 128u * (uint32_t)s, qtr);
                 const int a0 = (pw < 4) ? 0 : 4, a1 = min(nak, a0 + 4);
-                for (int at = a0; at < a1; ++at) {
-                    float v[16];
-                    tmem_ld16(eq + 16u * at, v);
-                    tmem_wait_ld();
+                tmem_pieces<1>(eq + 16u * (uint32_t)a0, a1 - a0, [&](int j0, float (&v)[16]) {
+                    const int at = a0 + j0;
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] = -v[j];
                     const uint32_t wa = stg + (uint32_t)at * kAtomKQW + kAtW;
@@ -714,17 +765,26 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] = 0.0f;
                     tmem_st16(eq + 16u * at, v);
-                }
+                });
                 tmem_wait_st();
             }
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(kBarPrep, kPrepThreads);
             if (pt == 0) mbar_arrive(bar(B_READY + s));
+            return true;
+        };
+        for (Cursor cu(a, P, warm0); ok && cu.valid(); cu.next()) {
+            ok = front(cu);
+            if (!ok) break;
+            inverse_t(cu.n & 1);
+            ok = back(cu.n);
         }
     } else {
-        // ======================= chain and output (warps 12-15) =======================
-        const int q = warp - kChainWarp0, row = 32 * q + lane;
+        // ======================= chain and output (warps 12-19) =======================
+        const int q = cq, row = 32 * q + lane;
+        const uint32_t a_lo = (uint32_t)c_alo;
+        const int na = c_na;
         bool ok = true;
         for (Cursor cu(a, P, warm0); cu.valid(); cu.next()) {
             const int n = cu.n, s = n & 1, L = cu.L();
@@ -733,8 +793,6 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (cu.first() && n > 0) chain_init(pc);
             const uint32_t eqs = tlane(tmem + kColEQS + 128u * (uint32_t)s, q);
             const float* cs = reinterpret_cast<const float*>(gb + (uint32_t)s * kStageBytes + kStageSc);
-            // decay of the next chunk of this piece, applied to the state when it is read back
-            const float gl_next = last ? 1.0f : __expf(-chunk_decay(p, pc.b, pc.h, cu.c + 1, lane));
             ok = mbar_wait(bar(B_READY + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 51);
             ok = ok && mbar_wait(bar(B_M1), (uint32_t)(n & 1), abort_flag, lim, 52);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -743,25 +801,28 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // E (TMEM lanes 64-127): E' = diag(e^{G_L-G}/|k|) E for MMA2, then E for P E
                 const int i = row - 64;
                 const float dl = cs[CS_DL + i];
-                for (int at = 0; at < nav; ++at) {
-                    float v[16];
-                    tmem_ld16(eqs + 16u * at, v);
-                    tmem_wait_ld();
+                tmem_pieces<1>(eqs + 16u * a_lo, na, [&](int j0, float (&v)[16]) {
+                    const uint32_t at = a_lo + (uint32_t)j0;
+                    float e[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] *= dl;
-                    st_bf16x8(sw32_at(base + kOffEp, kAtomE, (uint32_t)i, 16u * at), &v[0]);
-                    st_bf16x8(sw32_at(base + kOffEp, kAtomE, (uint32_t)i, 16u * at + 8u), &v[8]);
-                }
+                    for (int j = 0; j < 16; ++j) e[j] = v[j] * dl;
+                    st_bf16x8(sw32_at(base + kOffEp, kAtomE, (uint32_t)i, 16u * at), &e[0]);
+                    st_bf16x8(sw32_at(base + kOffEp, kAtomE, (uint32_t)i, 16u * at + 8u), &e[8]);
+                });
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_EREADY));
-                for (int at = 0; at < nav; ++at) {
-                    float v[16];
-                    tmem_ld16(eqs + 16u * at, v);
-                    tmem_wait_ld();
+                // (the E tile doubles as the previous chunk's output staging: wait for its store)
+                if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(B_OFREE), (uint32_t)((n - 1) & 1), abort_flag,
+                                                                 lim, 57))) {
+                    ok = false;
+                    break;
+                }
+                tmem_pieces<1>(eqs + 16u * a_lo, na, [&](int j0, float (&v)[16]) {
+                    const uint32_t at = a_lo + (uint32_t)j0;
                     st_bf16x8(sw32_at(base + kOffE, kAtomE, (uint32_t)i, 16u * at), &v[0]);
                     st_bf16x8(sw32_at(base + kOffE, kAtomE, (uint32_t)i, 16u * at + 8u), &v[8]);
-                }
+                });
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
@@ -769,21 +830,27 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             } else {
                 // Q S (TMEM lanes 0-63) scaled in place by e^G/|q|; P E is added onto it
                 const float gq = cs[CS_GQ + row];
-                for (int at = 0; at < nav; ++at) {
-                    float v[16];
-                    tmem_ld16(eqs + 16u * at, v);
-                    tmem_wait_ld();
+                tmem_pieces<1>(eqs + 16u * a_lo, na, [&](int j0, float (&v)[16]) {
+                    const uint32_t at = a_lo + (uint32_t)j0;
 #pragma unroll
                     for (int j = 0; j < 16; ++j) v[j] *= gq;
                     tmem_st16(eqs + 16u * at, v);
-                }
+                });
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_PEGO));
             }
             // ---- next state: bf16 copy for MMA1, decayed fp32 back into SACC ----
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_M2), (uint32_t)(n & 1), abort_flag, lim, 53));
+            // decay of the next chunk of this piece (its stage's gates), applied to the state
+            // when it is read back
+            float gl_next = 1.0f;
+            if (!last) {
+                ok = mbar_wait(bar(B_FULL + ((n + 1) & 1)), (uint32_t)(((n + 1) >> 1) & 1), abort_flag, lim, 55);
+                gl_next = reinterpret_cast<const float*>(gb + (uint32_t)((n + 1) & 1) * kStageBytes + kStageSc)[CS_GL];
+            }
+            ok = ok && mbar_wait(bar(B_M2), (uint32_t)(n & 1), abort_flag, lim, 53);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
             {
@@ -791,10 +858,8 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 float* so = (last && pc.wr && row < dk)
                                 ? p.state_out + (((size_t)pc.b * p.H + pc.h) * dk + row) * (size_t)dv
                                 : nullptr;
-                for (int at = 0; at < nav; ++at) {
-                    float v[16];
-                    tmem_ld16(sa + 16u * at, v);
-                    tmem_wait_ld();
+                tmem_pieces<1>(sa + 16u * a_lo, na, [&](int j0, float (&v)[16]) {
+                    const uint32_t at = a_lo + (uint32_t)j0;
                     if (so) {
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
@@ -810,7 +875,7 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         for (int j = 0; j < 16; ++j) v[j] *= gl_next;
                         tmem_st16(sa + 16u * at, v);
                     }
-                }
+                });
                 if (!last) {
                     tmem_wait_st();
                     fence_proxy_async_smem();
@@ -819,30 +884,37 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (lane == 0) mbar_arrive(bar(B_SREADY));
                 }
             }
-            // ---- output rows (TMEM lanes 0-63) ----
+            // ---- output rows (TMEM lanes 0-63): bf16 rows into the E tile, one TMA store ----
             if (q < 2) {
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEDONE), (uint32_t)(n & 1), abort_flag, lim, 54));
                 if (!ok) break;
                 tc_fence_after();
-                if (emit && p.out) {
-                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) +
-                                       (((size_t)pc.b * p.T + (size_t)cu.c * kC + row) * p.H + pc.h) * dv;
-                    for (int at = 0; at < nav; ++at) {
-                        float v[16];
-                        tmem_ld16(eqs + 16u * at, v);
-                        tmem_wait_ld();
-                        if (row < L) {
-                            uint4* o4 = reinterpret_cast<uint4*>(o + 16 * at);
-                            o4[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                               pack_bf16x2(v[6], v[7]));
-                            o4[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
-                                               pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
-                        }
-                    }
+                const bool store = emit && p.out != nullptr;
+                if (store) {
+                    const uint32_t orow = base + kOffE + (uint32_t)row * (uint32_t)(2 * dv);
+                    tmem_pieces<1>(eqs + 16u * a_lo, na, [&](int j0, float (&v)[16]) {
+                        const uint32_t at = a_lo + (uint32_t)j0;
+                        st_shared_v4(orow + 32u * at, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                     pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                        st_shared_v4(orow + 32u * at + 16u, pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                                     pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+                    });
+                    fence_proxy_async_smem();
                 }
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_EQFREE + s));
+                named_bar_sync(kBarOut, 128);
+                if (warp == kChainWarp0) {
+                    if (lane == 0) {
+                        if (store) {
+                            tma_store_4d(&tm_o, base + kOffE, 0, pc.h, cu.c * kC, pc.b);
+                            bulk_commit_group();
+                            bulk_wait_group_read0();
+                        }
+                        mbar_arrive_relaxed(bar(B_OFREE));
+                        mbar_arrive_relaxed(bar(B_EQFREE + s));
+                    }
+                    __syncwarp();
+                }
             }
         }
     }
@@ -879,9 +951,16 @@ cudaError_t launch_seq(const FwdParams& p, cudaStream_t stream)
     const long long nc = (p.T + seq::kC - 1) / seq::kC;
     const long long U = (long long)p.B * p.H * nc;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, p.q, p.dk, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
-        !make_map(&mk, p.k, p.dk, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
-        !make_map(&mv, p.v, p.dv, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B))
+    // 32-byte boxes, each read by exactly one CTA: no L2 promotion, so that a box
+    // fetches its own sectors only and not the neighbouring heads' bytes
+    const CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_NONE;
+    CUtensorMap mo;
+    if (!make_map(&mq, p.q, p.dk, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B, promo) ||
+        !make_map(&mk, p.k, p.dk, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B, promo) ||
+        !make_map(&mv, p.v, p.dv, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B, promo))
+        return cudaErrorInvalidValue;
+    // output: whole 64-token rows of d_v per store (no swizzle); the q map stands in when there is no output
+    if (p.out ? !make_map(&mo, p.out, p.dv, p.H, p.T, p.B, p.dv, CU_TENSOR_MAP_SWIZZLE_NONE, promo) : (mo = mq, false))
         return cudaErrorInvalidValue;
     seq::SeqArgs args;
     args.p = p;
@@ -898,7 +977,7 @@ cudaError_t launch_seq(const FwdParams& p, cudaStream_t stream)
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = args.grid_sync ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, seq::gdn_seq_kernel, mq, mk, mv, args);
+    return cudaLaunchKernelEx(&cfg, seq::gdn_seq_kernel, mq, mk, mv, mo, args);
 }
 
 }  // namespace gdn

@@ -814,7 +814,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 
 // 4-D bf16 map over a [B, T, H, inner] tensor, box {box_inner, 1, 64, 1}.
 bool make_map(CUtensorMap* map, const void* base, int inner, int H, int T, int B, int box_inner,
-              CUtensorMapSwizzle swz)
+              CUtensorMapSwizzle swz, CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B)
 {
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
     if (!fn) return false;
@@ -824,8 +824,7 @@ bool make_map(CUtensorMap* map, const void* base, int inner, int H, int T, int B
     cuuint32_t box[4] = {(cuuint32_t)box_inner, 1, (cuuint32_t)tc::kC, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // 2 s
