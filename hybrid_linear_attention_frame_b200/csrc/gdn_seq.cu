@@ -56,7 +56,6 @@ constexpr int kWarpLoadKQ = 0, kWarpGram = 1, kWarpChainMma = 2, kWarpWU = 3;
 constexpr int kPrepWarp0 = 4, kChainWarp0 = 12;
 constexpr int kPrepThreads = 256;
 constexpr uint32_t kBarPrep = 1;             // named barrier of the prep warps (3: the UT inverse's)
-constexpr uint32_t kBarOut = 2;              // named barrier of the four output warps
 constexpr uint32_t kBarA = 4;                // the four prep warps that form A and invert I + A
 
 // product of gates over a warm-up stretch below which the state entering it is dropped: 2^-48
@@ -110,7 +109,8 @@ enum : uint32_t {
     B_M2 = 18,        // MMA2 done
     B_PEDONE = 19,    // P E done
     B_OFREE = 20,     // output staging (the E tile) read by its TMA store
-    kNumBars = 21,
+    B_OREADY = 21,    // the four output warps' rows staged
+    kNumBars = 22,
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
@@ -147,7 +147,10 @@ static_assert(kOffAXI % 16 == 0 && kOffSc % 16 == 0 && kOffBar % 8 == 0, "alignm
 constexpr uint32_t kIdGram = idesc_bf16(128, 128, false, false);
 
 __host__ __device__ constexpr uint32_t bar_count(uint32_t i) {
-    return (i == B_SREADY || i == B_PEGO) ? 8u : (i == B_EREADY) ? 4u : (i == B_FULL || i == B_FULL + 1) ? 2u : 1u;
+    return (i == B_SREADY || i == B_PEGO) ? 8u
+           : (i == B_EREADY || i == B_OREADY) ? 4u
+           : (i == B_FULL || i == B_FULL + 1) ? 2u
+                                              : 1u;
 }
 
 // descriptors: K-major / MN-major 32-byte swizzle (8-row groups 256 B apart), K-major 128-byte swizzle
@@ -654,54 +657,79 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             return true;
         };
         // A (fp32, transposed above the diagonal of AXI; TMEM lanes 0-63) and P (bf16
-        // tile P[s]; lanes 64-127) from the Gram, row 32 (qtr & 1) + lane of each warp.
+        // tile P[s]; lanes 64-127) from the Gram, row i = 32 (qtr & 1) + lane of each warp,
+        // one 16-column block j0 = 16 bj at a time.  For a row in a later 16-row block
+        // than the columns (bi > bj) the decay factors through the block boundary,
+        // e^{G_i - G_j} = e^{G_i - G_{16 bi - 1}} e^{G_{16 bi - 1} - G_j} (both factors <= 1);
+        // inside the diagonal block it is one exponential; above it A has nothing and P is 0.
+        // Each warp takes two column blocks, chosen so that the costly diagonal blocks of
+        // a row group fall on different warps.
         auto gram_epilogue = [&](int s) {
-            {
-                const uint32_t ptile = base + kOffP + kTile * (uint32_t)s;
-                const int ch = pw >> 2;
-                if ((qtr & 1) == 0 && ch == 1) {
-                    // rows 0-31 x columns 32-63 lie above the diagonal: A has nothing there, P is zero
-                    if (qtr == 2) {
-                        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            const uint32_t ptile = base + kOffP + kTile * (uint32_t)s;
+            const bool isA = qtr < 2;
+            const int i = 32 * (qtr & 1) + lane, bi = i >> 4, ii = i & 15, ch = pw >> 2;
+            const int bmax = 2 * (qtr & 1) + 1;       // the warp's rows lie in blocks bmax - 1, bmax
+            const float Gi = sc[SC_G + i];
+            const float R = isA ? sc[SC_BETA + i] * sc[SC_RK + i] : sc[SC_RQ + i];
+            const float RX = R * sc[SC_EXR + i];
+#pragma unroll 1
+            for (int pc = 0; pc < 2; ++pc) {
+                const int bj = pc == 0 ? ch : ((qtr & 1) ? 3 - ch : 2 + ch);
+                const int j0 = 16 * bj;
+                float v[16];
+                if (bj > bmax) {
+                    // above the diagonal for every row of the warp
+                    if (!isA) {
 #pragma unroll
-                        for (int g8 = 0; g8 < 4; ++g8) st_bf16x8(ptile + sw128_offset((uint32_t)lane, 32u + 8u * g8), z);
+                        for (int jj = 0; jj < 16; ++jj) v[jj] = 0.0f;
+                        st_bf16x8(ptile + sw128_offset((uint32_t)i, (uint32_t)j0), &v[0]);
+                        st_bf16x8(ptile + sw128_offset((uint32_t)i, (uint32_t)j0 + 8u), &v[8]);
+                    }
+                    continue;
+                }
+                tmem_ld16(tlane(tg, qtr) + (uint32_t)j0, v);
+                tmem_wait_ld();
+                if (bi > bj) {
+                    const float* rk = sc + SC_RK + j0;
+                    const float* ex = sc + SC_EXC + 64 * bi + j0;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 r4 = ld4(rk + 4 * q4), e4 = ld4(ex + 4 * q4);
+                        v[4 * q4] *= RX * (r4.x * e4.x);
+                        v[4 * q4 + 1] *= RX * (r4.y * e4.y);
+                        v[4 * q4 + 2] *= RX * (r4.z * e4.z);
+                        v[4 * q4 + 3] *= RX * (r4.w * e4.w);
+                    }
+                } else if (bi == bj) {
+                    const float* rk = sc + SC_RK + j0;
+                    const float* gj = sc + SC_G + j0;
+                    const int lim_j = isA ? ii : ii + 1;       // A: j < i, P: j <= i
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 r4 = ld4(rk + 4 * q4), g4 = ld4(gj + 4 * q4);
+                        const float rr[4] = {r4.x, r4.y, r4.z, r4.w}, gg[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int jj = 4 * q4 + e;
+                            const float x = v[jj] * (R * rr[e]) * __expf(Gi - gg[e]);
+                            v[jj] = (jj < lim_j) ? x : 0.0f;
+                        }
                     }
                 } else {
-                    const int i = 32 * (qtr & 1) + lane;
-                    const int bi = i >> 4;
-                    const float Gi = sc[SC_G + i], exr = sc[SC_EXR + i];
-                    const float ri = (qtr < 2) ? sc[SC_BETA + i] * sc[SC_RK + i] : sc[SC_RQ + i];
-#pragma unroll 1
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int j0 = 32 * ch + 16 * hh;
-                        float v[16], val[16];
-                        tmem_ld16(tlane(tg, qtr) + (uint32_t)j0, v);
-                        tmem_wait_ld();
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const float4 g4 = ld4(sc + SC_G + j0 + 4 * q4);
-                            const float4 r4 = ld4(sc + SC_RK + j0 + 4 * q4);
-                            const float4 e4 = ld4(sc + SC_EXC + 64 * bi + j0 + 4 * q4);
-                            const float gj[4] = {g4.x, g4.y, g4.z, g4.w};
-                            const float rkj[4] = {r4.x, r4.y, r4.z, r4.w};
-                            const float ex[4] = {e4.x, e4.y, e4.z, e4.w};
+                    for (int jj = 0; jj < 16; ++jj) v[jj] = 0.0f;
+                }
+                if (isA) {
+                    if (bi >= bj) {
+                        float* dst = AXI + j0 * kXS + i;
+                        const int n_st = (bi > bj) ? 16 : ii;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int jj = 4 * q4 + e, j = j0 + jj;
-                                const float dec = ((j >> 4) == bi) ? __expf(Gi - gj[e]) : exr * ex[e];
-                                const bool keep = (qtr < 2) ? (j < i) : (j <= i);
-                                val[jj] = keep ? ri * rkj[e] * v[jj] * dec : 0.0f;
-                            }
-                        }
-                        if (qtr < 2) {
-#pragma unroll
-                            for (int jj = 0; jj < 16; ++jj)
-                                if (j0 + jj < i) AXI[(j0 + jj) * kXS + i] = val[jj];
-                        } else {
-                            st_bf16x8(ptile + sw128_offset((uint32_t)i, (uint32_t)j0), &val[0]);
-                            st_bf16x8(ptile + sw128_offset((uint32_t)i, (uint32_t)j0 + 8u), &val[8]);
-                        }
+                        for (int jj = 0; jj < 16; ++jj)
+                            if (jj < n_st) dst[jj * kXS] = v[jj];
                     }
+                } else {
+                    st_bf16x8(ptile + sw128_offset((uint32_t)i, (uint32_t)j0), &v[0]);
+                    st_bf16x8(ptile + sw128_offset((uint32_t)i, (uint32_t)j0 + 8u), &v[8]);
                 }
             }
         };
@@ -901,9 +929,14 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     });
                     fence_proxy_async_smem();
                 }
+                // (an mbarrier rather than a named barrier: a warp that gave up on a wait
+                // never arrives, and the storing warp's wait for it is bounded)
                 tc_fence_before();
-                named_bar_sync(kBarOut, 128);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_OREADY));
                 if (warp == kChainWarp0) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OREADY), (uint32_t)(n & 1), abort_flag, lim, 58));
+                    if (!ok) break;
                     if (lane == 0) {
                         if (store) {
                             tma_store_4d(&tm_o, base + kOffE, 0, pc.h, cu.c * kC, pc.b);

@@ -64,6 +64,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of the phase (try_wait, even without a hint, may hold the thread
+// until the phase completes or a hardware-chosen time runs out).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // try_wait that may suspend the thread for up to `hint_ns` while the phase is
 // incomplete (it resumes as soon as the phase completes), so that waiting warps
 // leave issue slots to the warps sharing their scheduler.
@@ -83,15 +94,16 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
 // (first error wins) and returns false.
 // (The polling loop is an out-of-line function: waits are many and mostly
 // succeed at once, and inlining the loop everywhere bloats the code.)
-// Under a short bound (below 1 ms) the phase is polled without the suspend
-// hint and the clock read at every poll, so that the bound is observed even
-// when the phase completes within the hint's time.
+// Under a short bound (below 1 ms) the phase is polled with the non-blocking
+// test and the clock read at every poll, so that the bound is observed even when
+// the phase would complete within a blocking poll's time.
+constexpr uint64_t kShortBoundNs = 1000000ull;
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
                                             uint64_t limit_ns, int code) {
     const uint64_t t0 = globaltimer_ns();
-    const bool short_bound = limit_ns < 1000000ull;
+    const bool short_bound = limit_ns < kShortBoundNs;
     for (uint32_t it = 1;; ++it) {
-        if (short_bound ? mbar_try_wait(bar, parity) : mbar_try_wait_hint(bar, parity, 1000u)) return true;
+        if (short_bound ? mbar_test_wait(bar, parity) : mbar_try_wait_hint(bar, parity, 1000u)) return true;
         if (short_bound || (it & 63u) == 0) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
@@ -105,7 +117,7 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns, int code) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (limit_ns >= kShortBoundNs && mbar_try_wait(bar, parity)) return true;
     return mbar_wait_slow(bar, parity, abort, limit_ns, code);
 }
 

@@ -4,14 +4,14 @@ return, leaving the context usable.
 
 The test shortens the bound to 1 ns through gdn_set_wait_limit_ns, so that the
 first wait that does not succeed at once gives up (nothing is broken: the
-producer is simply slower than the bound).  In the ring kernel the copy warp that
-waits, on a shared-memory counter, for the first record of its group polls the
-clock every ~1 us, while that record takes several microseconds of tensor-core work
-to appear, so the call times out every time.  The fused kernel waits only on
-mbarriers with a suspend-time hint, and a hinted poll has been seen to return only
-once the phase completed, so its calls finish normally; either status is accepted
-there.  After each such call the default bound is restored and a
-normal call must match the untouched reference outputs bit for bit.
+producer is simply slower than the bound).  Under a bound below 1 ms the mbarrier
+waits poll without a suspend hint and read the clock on every poll, and the ring
+kernel's counter waits read it every ~1 us, so every kernel reports the timeout:
+the ring kernel (gdn_forward_ws), the sequence-parallel kernel (gdn_forward at
+d 112) and the fused chunk kernel (gdn_forward at d 128).  Each kernel then
+drains the copies and MMAs it has in flight and returns.  After each such call
+the default bound is restored and a normal call must match the untouched
+reference outputs bit for bit.
 """
 
 import numpy as np
@@ -24,10 +24,10 @@ from gpu_util import f32_device, upload
 pytestmark = pytest.mark.gpu
 
 
-def _inputs():
+def _inputs(d):
     rng = np.random.Generator(np.random.PCG64(77))
-    # 2 x 20 chains of 700 tokens at d 112: a ring of 7 x 20 CTAs
-    return draw(rng, 2, 20, 700, 112, 112, 100, "bf16", gate_mean=0.0, gate_std=1.5, state_std=0.3)
+    # 2 x 20 chains of 700 tokens (at d 112 a ring of 7 x 20 CTAs)
+    return draw(rng, 2, 20, 700, d, d, 100, "bf16", gate_mean=0.0, gate_std=1.5, state_std=0.3)
 
 
 def _run(G, entry, tensors, inp, ws):
@@ -44,11 +44,14 @@ def _run(G, entry, tensors, inp, ws):
     return o, s, G.gdn_get_last_device_status()
 
 
-@pytest.mark.parametrize("entry", ["ws", "plain"])
-def test_wait_timeout_is_reported_and_context_recovers(cuda, entry):
+@pytest.mark.parametrize("entry,d,path", [("ws", 112, None), ("plain", 112, 2), ("plain", 128, 1)],
+                         ids=["ring", "sequence_parallel", "fused_d128"])
+def test_wait_timeout_is_reported_and_context_recovers(cuda, entry, d, path):
     import torch
     import hybrid_linear_attention_frame_b200 as G
-    inp = _inputs()
+    if path is not None:
+        assert G.gdn_bf16_path(d, d, 64) == path
+    inp = _inputs(d)
     q, k, v, g, b = upload(inp, cuda)
     s_in = f32_device(inp.state, cuda)
     Bn, T, H, dk = inp.q.shape
@@ -63,10 +66,7 @@ def test_wait_timeout_is_reported_and_context_recovers(cuda, entry):
         assert G.gdn_set_wait_limit_ns(1) == G.GDN_OK
         for _ in range(3):
             _, _, st = _run(G, entry, tensors, inp, ws)
-            if entry == "ws":
-                assert st == G.GDN_ERR_TIMEOUT, G.status_string(st)
-            else:
-                assert st in (G.GDN_OK, G.GDN_ERR_TIMEOUT), G.status_string(st)
+            assert st == G.GDN_ERR_TIMEOUT, G.status_string(st)
             print(f"{entry}: status under a 1 ns bound: {G.status_string(st)}")
     finally:
         G.gdn_set_wait_limit_ns(0)
