@@ -22,8 +22,8 @@
 //   prep  Gram  [K;Q][K;Q]^T            -> norms (diagonal), A and P with the decay
 //         T = (I+A)^{-1} diag(beta), T' = T diag(e^G/|k|)  (CUDA cores + mma.sync)
 //         U = [Z;T] V, then W = [T';Z] K accumulated  -> EQS = [W ; U]
-//         -W to shared memory beside Q; lanes 0-63 of EQS cleared  -> EQS = [0 ; U]
-//   chain MMA1  [Q;-W] S_bf16 onto EQS   -> [Q S ; E = U - W S]
+//   chain -W to shared memory beside Q; lanes 0-63 of EQS cleared  -> EQS = [0 ; U]
+//         MMA1  [Q;-W] S_bf16 onto EQS   -> [Q S ; E = U - W S]
 //         E' = diag(e^{G_L-G}/|k|) E and E in bf16;  Q S scaled by e^G/|q| in TMEM
 //         MMA2  K^T E' onto SACC = e^{G_L} S  -> next state (fp32, in TMEM)
 //         PE    [P;X] E onto EQS lanes 0-63   -> O = diag(e^G/|q|) Q S + P E
@@ -57,6 +57,7 @@ constexpr int kPrepWarp0 = 4, kChainWarp0 = 12;
 constexpr int kPrepThreads = 256;
 constexpr uint32_t kBarPrep = 1;             // named barrier of the prep warps (3: the UT inverse's)
 constexpr uint32_t kBarA = 4;                // the four prep warps that form A and invert I + A
+constexpr uint32_t kBarP = 5;                // the four prep warps that form P
 
 // product of gates over a warm-up stretch below which the state entering it is dropped: 2^-48
 constexpr float kWarmupLogDecay = 48.0f * 0.693147181f;
@@ -90,27 +91,30 @@ constexpr uint32_t kOffE = kOffEp + kMaxAtoms * kAtomE;      // E bf16; then the
 constexpr uint32_t kOffAXI = kOffE + kMaxAtoms * kAtomE;     // fp32 [64][kXS]: A / (I+A)^{-1}
 constexpr uint32_t kScFloats = 13 * 64 + 16;
 constexpr uint32_t kOffSc = kOffAXI + 64 * kXS * 4;          // prep scalar table
-constexpr uint32_t kOffBar = kOffSc + kScFloats * 4;
+constexpr uint32_t kOffMS = kOffSc + kScFloats * 4;         // the UT inverse's scratch
+constexpr uint32_t kMSBytes = 4 * tc::kMS * 32 * 4;
+constexpr uint32_t kOffBar = kOffMS + kMSBytes;
 enum : uint32_t {
     B_FULL = 0,       // [2] q/k tiles of a stage landed and its gates written
     B_SFREE = 2,      // [2] chain MMAs done with a stage (and with its P)
     B_VFULL = 4,      // v tile landed
     B_VFREE = 5,      // U MMA done with the v tile
     B_G1 = 6,         // Gram done
-    B_GFREE = 7,      // Gram read by the prep
+    B_GFREE = 7,      // Gram read by the prep (A and P warp groups)
     B_TREADY = 8,     // T' and T written
-    B_WU = 9,         // U and W MMAs done
-    B_READY = 10,     // [2] stage complete for the chain (-W written, EQS = [0;U], scalars)
-    B_EQFREE = 12,    // [2] output read from EQS
-    B_SREADY = 14,    // bf16 state written and SACC decayed
-    B_M1 = 15,        // MMA1 done
-    B_EREADY = 16,    // E' written
-    B_PEGO = 17,      // E written and Q S scaled
-    B_M2 = 18,        // MMA2 done
-    B_PEDONE = 19,    // P E done
-    B_OFREE = 20,     // output staging (the E tile) read by its TMA store
-    B_OREADY = 21,    // the four output warps' rows staged
-    kNumBars = 22,
+    B_WU = 9,         // [2] U and W MMAs of a stage done
+    B_READY = 11,     // [2] the prep done with a stage (P, scalars, T read by the U/W MMAs)
+    B_EQFREE = 13,    // [2] output read from EQS
+    B_SREADY = 15,    // bf16 state written and SACC decayed
+    B_M1 = 16,        // MMA1 done
+    B_EREADY = 17,    // E' written
+    B_PEGO = 18,      // E written and Q S scaled
+    B_M2 = 19,        // MMA2 done
+    B_PEDONE = 20,    // P E done
+    B_OFREE = 21,     // output staging (the E tile) read by its TMA store
+    B_OREADY = 22,    // the four output warps' rows staged
+    B_WREADY = 23,    // -W written beside Q and EQS lanes 0-63 cleared (four chain warps)
+    kNumBars = 24,
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
@@ -141,16 +145,15 @@ static_assert(kOffP % 1024 == 0 && kOffTp % 1024 == 0 && kStageBytes % 1024 == 0
 static_assert(kOffS % 256 == 0 && kOffEp % 256 == 0 && kOffE % 256 == 0 && kOffV % 256 == 0 &&
                   kAtomKQW % 256 == 0 && kAtomS % 256 == 0,
               "SW32 alignment");
-static_assert(4 * tc::kMS * 32 * 4 <= kTile, "solve scratch fits in the T tile");
-static_assert(kOffAXI % 16 == 0 && kOffSc % 16 == 0 && kOffBar % 8 == 0, "alignment");
+static_assert(kOffAXI % 16 == 0 && kOffSc % 16 == 0 && kOffMS % 16 == 0 && kOffBar % 8 == 0, "alignment");
 
 constexpr uint32_t kIdGram = idesc_bf16(128, 128, false, false);
 
 __host__ __device__ constexpr uint32_t bar_count(uint32_t i) {
     return (i == B_SREADY || i == B_PEGO) ? 8u
-           : (i == B_EREADY || i == B_OREADY) ? 4u
-           : (i == B_FULL || i == B_FULL + 1) ? 2u
-                                              : 1u;
+           : (i == B_EREADY || i == B_OREADY || i == B_WREADY) ? 4u
+           : (i == B_FULL || i == B_FULL + 1 || i == B_GFREE) ? 2u
+                                                               : 1u;
 }
 
 // descriptors: K-major / MN-major 32-byte swizzle (8-row groups 256 B apart), K-major 128-byte swizzle
@@ -537,7 +540,7 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int ks = 0; ks < kC / 16; ++ks)   // + [T';Z] K -> [W ; U]
                 mma_bf16_warp(eqs, dk128(base + kOffTp + 32u * ks), dmn32(st + 512u * ks, kAtomKQW), idw, 1u);
-            mma_commit_warp(bar(B_WU));
+            mma_commit_warp(bar(B_WU + (uint32_t)s));
             mma_commit_warp(bar(B_VFREE));
             wu_issued = n + 1;
             cv.next();
@@ -550,7 +553,8 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
         if (!ok && lane == 0) {
-            if (wu_issued > 0) drain_wait(bar(B_WU), (uint32_t)((wu_issued - 1) & 1));
+            if (wu_issued > 0)
+                drain_wait(bar(B_WU + (uint32_t)((wu_issued - 1) & 1)), (uint32_t)(((wu_issued - 1) >> 1) & 1));
             if (v_issued > wu_issued) drain_wait(bar(B_VFULL), (uint32_t)((v_issued - 1) & 1));
         }
         __syncwarp();
@@ -564,6 +568,7 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t eqs = tmem + kColEQS + 128u * (uint32_t)s;
             const uint32_t st = base + (uint32_t)s * kStageBytes;
             ok = mbar_wait(bar(B_READY + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 31);
+            ok = ok && mbar_wait(bar(B_WREADY), (uint32_t)(n & 1), abort_flag, lim, 35);
             ok = ok && mbar_wait(bar(B_SREADY), (uint32_t)(n & 1), abort_flag, lim, 32);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
@@ -600,11 +605,11 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int pt = tid - kPrepWarp0 * 32, pw = warp - kPrepWarp0;
         float* sc = reinterpret_cast<float*>(gb + kOffSc);
         float* AXI = reinterpret_cast<float*>(gb + kOffAXI);
-        float* MSf = reinterpret_cast<float*>(gb + kOffT);
+        float* MSf = reinterpret_cast<float*>(gb + kOffMS);
         const uint32_t tg = tmem + kColG;
         bool ok = true;
-        // Per chunk: front (the stage's gates, norms, A and P from the Gram), the UT
-        // inverse and T, T', then back (-W beside Q once the U and W MMAs are done).
+        // Per chunk: front (the stage's gates, norms), then A and P from the Gram, the
+        // UT inverse and T, T'.
         auto front = [&](const Cursor& cu) -> bool {
             const int n = cu.n, s = n & 1, L = cu.L();
             float* cs = reinterpret_cast<float*>(gb + (uint32_t)s * kStageBytes + kStageSc);
@@ -734,16 +739,26 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         };
         // The warps on TMEM lanes 0-63 (qtr 0, 1) form A and then invert I + A; the
-        // warps on lanes 64-127 form P meanwhile (P is needed only by the chain).
-        auto inverse_t = [&](int s) {
+        // warps on lanes 64-127 form P meanwhile (P is needed only by the chain).  Each
+        // group releases its half of the Gram accumulator as soon as it has read it.
+        // T and T' are written once the previous chunk's U/W MMAs have read them; the
+        // chain warps then take -W out of TMEM, so the prep goes straight on to the
+        // next chunk.
+        auto inverse_t = [&](int n) -> bool {
+            const int s = n & 1;
             gram_epilogue(s);
+            tc_fence_before();
             if (qtr < 2) {
                 named_bar_sync(kBarA, 128);      // A complete
+                if (pw == 0 && lane == 0) mbar_arrive(bar(B_GFREE));
                 tc::unit_lower_inverse_64(AXI, MSf, 32 * ((pw & 1) | ((pw >> 2) << 1)) + lane);
+            } else {
+                named_bar_sync(kBarP, 128);      // P complete
+                if (pw == 2 && lane == 0) mbar_arrive(bar(B_GFREE));
             }
-            tc_fence_before();
-            named_bar_sync(kBarPrep, kPrepThreads);
-            if (pt == 0) mbar_arrive(bar(B_GFREE));       // the Gram accumulator may be overwritten
+            bool okw = true;
+            if (n > 0) okw = mbar_wait(bar(B_WU + (uint32_t)((n - 1) & 1)), (uint32_t)(((n - 1) >> 1) & 1), abort_flag, lim, 42);
+            if (!group_all(kBarPrep, kPrepThreads, okw)) return false;
             // ---- T = (I+A)^{-1} diag(beta), T' = T diag(beta e^G / |k|): bf16 tiles ----
             {
                 const int i = pt >> 2, jb = 16 * (pt & 3);
@@ -770,49 +785,24 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             fence_proxy_async_smem();
             named_bar_sync(kBarPrep, kPrepThreads);
-            if (pt == 0) mbar_arrive(bar(B_TREADY));
-        };
-        auto back = [&](int n) -> bool {
-            const int s = n & 1;
-            const uint32_t stg = base + (uint32_t)s * kStageBytes;
-            // ---- U and W done: -W beside Q, then clear lanes 0-63 of EQS ----
-            ok = mbar_wait(bar(B_WU), (uint32_t)(n & 1), abort_flag, lim, 42);
-            if (!group_all(kBarPrep, kPrepThreads, ok)) return false;
-            tc_fence_after();
-            if (qtr < 2) {
-                const int i = 32 * qtr + lane;
-                const uint32_t eq = tlane(tmem + kColEQS + 128u * (uint32_t)s, qtr);
-                const int a0 = (pw < 4) ? 0 : 4, a1 = min(nak, a0 + 4);
-                tmem_pieces<1>(eq + 16u * (uint32_t)a0, a1 - a0, [&](int j0, float (&v)[16]) {
-                    const int at = a0 + j0;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] = -v[j];
-                    const uint32_t wa = stg + (uint32_t)at * kAtomKQW + kAtW;
-                    st_bf16x8(wa + sw32_chunk_offset((uint32_t)i, 0), &v[0]);
-                    st_bf16x8(wa + sw32_chunk_offset((uint32_t)i, 1), &v[8]);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-                    tmem_st16(eq + 16u * at, v);
-                });
-                tmem_wait_st();
+            if (pt == 0) {
+                mbar_arrive(bar(B_TREADY));
+                mbar_arrive(bar(B_READY + s));
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar_sync(kBarPrep, kPrepThreads);
-            if (pt == 0) mbar_arrive(bar(B_READY + s));
             return true;
         };
         for (Cursor cu(a, P, warm0); ok && cu.valid(); cu.next()) {
             ok = front(cu);
             if (!ok) break;
-            inverse_t(cu.n & 1);
-            ok = back(cu.n);
+            ok = inverse_t(cu.n);
         }
     } else {
         // ======================= chain and output (warps 12-19) =======================
         const int q = cq, row = 32 * q + lane;
         const uint32_t a_lo = (uint32_t)c_alo;
         const int na = c_na;
+        // the half of the d_k atoms of W this warp takes out of TMEM (lane quarters 0, 1)
+        const int k_lo = chf ? (nak + 1) / 2 : 0, k_na = chf ? nak - (nak + 1) / 2 : (nak + 1) / 2;
         bool ok = true;
         for (Cursor cu(a, P, warm0); cu.valid(); cu.next()) {
             const int n = cu.n, s = n & 1, L = cu.L();
@@ -822,6 +812,30 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t eqs = tlane(tmem + kColEQS + 128u * (uint32_t)s, q);
             const float* cs = reinterpret_cast<const float*>(gb + (uint32_t)s * kStageBytes + kStageSc);
             ok = mbar_wait(bar(B_READY + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 51);
+            if (q < 2) {
+                // U and W done: -W (TMEM lanes 0-63 of EQS) beside Q in the stage, and
+                // those lanes cleared, so that MMA1 adds Q S onto zero
+                ok = ok && mbar_wait(bar(B_WU + (uint32_t)s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 56);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t stg = base + (uint32_t)s * kStageBytes;
+                tmem_pieces<1>(eqs + 16u * (uint32_t)k_lo, k_na, [&](int j0, float (&v)[16]) {
+                    const uint32_t at = (uint32_t)(k_lo + j0);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = -v[j];
+                    const uint32_t wa = stg + at * kAtomKQW + kAtW;
+                    st_bf16x8(wa + sw32_chunk_offset((uint32_t)row, 0), &v[0]);
+                    st_bf16x8(wa + sw32_chunk_offset((uint32_t)row, 1), &v[8]);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+                    tmem_st16(eqs + 16u * at, v);
+                });
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_WREADY));
+            }
             ok = ok && mbar_wait(bar(B_M1), (uint32_t)(n & 1), abort_flag, lim, 52);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
