@@ -588,8 +588,8 @@ def run_ours(args, w, rank, world, local):
     dims = (w.B, w.H, w.T, w.d_k, w.d_v, w.frame_len, w.chunk_len)
     bidir = args.direction == "bidir"
     gate_mode = 1 if args.gate_mode == "frame" else 0
-    if bidir and (gate_mode or args.path == "plain" or w.name != "minute"):
-        raise SystemExit("--direction bidir: minute workload, gate at every token, --path ws")
+    if bidir and (gate_mode or w.name != "minute"):
+        raise SystemExit("--direction bidir: minute workload, gate at every token")
     if gate_mode and stream_step:
         raise SystemExit("--gate-mode frame applies to the layer workloads")
     use_ws = args.path == "ws" and G.gdn_workspace_bytes(*dims[:5], w.chunk_len) > 0
@@ -672,7 +672,9 @@ def run_ours(args, w, rank, world, local):
     achieved = abytes / avg_launch_s / 1e9
     traffic, traffic_kernel = recorded_traffic()
     if bidir:
-        kernel = "gdn_forward_bidir (one layer call: reverse copy, 2 x gdn_ring_kernel, combine)"
+        kernel = ("gdn_forward_bidir (one layer call: reverse copy, 2 x "
+                  + ("gdn_seq_kernel" if G.gdn_bf16_path(w.d_k, w.d_v, w.chunk_len) == 2 else "gdn_ring_kernel")
+                  + ", combine)")
     elif use_ws:
         kernel = "gdn_ring_kernel"
     elif G.gdn_bf16_path(w.d_k, w.d_v, w.chunk_len) == 2:

@@ -132,7 +132,8 @@ int run_bf16_ws(const gdn::FwdParams& p, int chunk_len, void* ws, size_t ws_byte
 int bidir_need(int B, int H, int T, int dk, int dv, int chunk_len, size_t elem, gdn::BidirLayout* L)
 {
     size_t ring = 0;
-    if (elem == 2 && uses_ring(T, dk, dv, chunk_len)) {
+    // the two scans take the sequence-parallel kernel where it applies (no ring workspace)
+    if (elem == 2 && uses_ring(T, dk, dv, chunk_len) && !gdn::seq_supported(dk, dv, chunk_len)) {
         const int st = workspace_need(B, H, dv, &ring);
         if (st != GDN_OK) return st;
     }

@@ -259,14 +259,15 @@ int gdn_forward_gated_f32(const float* q, const float* k, const float* v,
  * aligned, not overlapping any argument, contents need no initialisation, owned by
  * the caller and busy until the call's work on `stream` completes) holds the
  * token-reversed copies of q, k, v, beta and the per-token gate logits, the backward
- * scan's output and, for the bf16 entry, the ring of gdn_forward_ws where those sizes
- * take it: gdn_bidir_workspace_bytes gives its size (about 1.5x the bytes of q, k
- * and v; 0 when T = 0).  elem_bytes is 2 for gdn_forward_bidir, 4 for
+ * scan's output and, for the bf16 entry at sizes that the sequence-parallel kernel
+ * does not take but the ring kernel of gdn_forward_ws does (d above 112), that
+ * ring: gdn_bidir_workspace_bytes gives its size (about 1.5x the bytes of q, k and
+ * v; 0 when T = 0).  elem_bytes is 2 for gdn_forward_bidir, 4 for
  * gdn_forward_bidir_f32.
  *
- * Work on `stream`: one copy kernel, the forward kernel twice (gdn_forward_ws's
- * ring kernel where it applies, else gdn_forward's; the float32 kernel of
- * gdn_forward_f32 for the _f32 entry), one combine kernel.  Rounding (bf16 entry):
+ * Work on `stream`: one copy kernel, the forward kernel twice (gdn_forward's
+ * kernel, or the ring kernel of gdn_forward_ws where the workspace holds a ring;
+ * the float32 kernel of gdn_forward_f32 for the _f32 entry), one combine kernel.  Rounding (bf16 entry):
  * each scan's output is rounded to bf16, their sum is formed in fp32 and rounded to
  * bf16 again.  Errors: as gdn_forward; a missing, misaligned, small or overlapping
  * workspace gives GDN_ERR_INVALID_ARG; B*T above 4 * INT32_MAX gives

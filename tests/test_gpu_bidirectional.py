@@ -3,8 +3,8 @@ against the float64 oracle's bidirectional form (forward scan plus backward scan
 from zero states, each token with its own frame's gate).  Bars: bf16 max-abs <= 2e-2
 and relative L2 <= 5e-3; float32 mode relative L2 <= 1e-4.
 
-Cases: sizes that take the ring kernel (d 112, ragged T, frames that do not divide
-T), the bf16 FFMA path (d 64 and 32, chunk 16/32/64), the float32 mode, single-token
+Cases: sizes that take the sequence-parallel kernel (d 112, ragged T, frames that
+do not divide T) and the ring kernel (d_v 128), the bf16 FFMA path (d 64 and 32, chunk 16/32/64), the float32 mode, single-token
 and sub-chunk sequences, more chains than CTA groups, the clip241 and minute-scale
 layers, and T = 0 (nothing is written).  Outputs are NaN-filled with guard bands,
 the workspace is filled with garbage first.
@@ -65,8 +65,8 @@ RNG_SEED = 31
 def cases_bf16():
     rng = np.random.Generator(np.random.PCG64(RNG_SEED))
     return {
-        "ring d112 ragged frames": (draw(rng, 2, 20, 700, 112, 112, 90, "bf16", 2.0, 0.5), 64),
-        "ring d112 strong decay": (draw(rng, 1, 4, 333, 112, 112, 50, "bf16", 0.0, 1.5), 64),
+        "seq d112 ragged frames": (draw(rng, 2, 20, 700, 112, 112, 90, "bf16", 2.0, 0.5), 64),
+        "seq d112 strong decay": (draw(rng, 1, 4, 333, 112, 112, 50, "bf16", 0.0, 1.5), 64),
         "ring d96 x 128": (draw(rng, 1, 6, 257, 96, 128, 64, "bf16", 1.0, 1.0), 64),
         "ffma d64": (draw(rng, 1, 3, 200, 64, 64, 50, "bf16", 0.0, 1.0), 64),
         "ffma d32 chunk 16": (draw(rng, 2, 2, 77, 32, 32, 7, "bf16", 0.5, 1.0), 16),
