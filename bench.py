@@ -80,6 +80,9 @@ def parse_args(argv=None):
     ap.add_argument("--direction", choices=["causal", "bidir"], default="causal",
                     help="causal: the forward scan; bidir: gdn_forward_bidir (forward plus backward "
                          "scan from zero states, the dense checkpoint's form)")
+    ap.add_argument("--inputs", choices=["bf16", "fp8"], default="bf16",
+                    help="bf16: q, k, v in bf16 (gdn_forward); fp8: q, k, v as e4m3 bytes, v with one "
+                         "power-of-two scale (gdn_forward_fp8; layer workloads, forward scan)")
     return ap.parse_args(argv)
 
 
@@ -192,11 +195,12 @@ class ClockSampler:
 # roofline bookkeeping
 # ----------------------------------------------------------------------------
 
-def algorithmic_bytes(w, state_in: bool, state_out: bool) -> int:
-    """Bytes one gdn_forward call must move at least: q, k, v, out (bf16), the
-    beta logits, the per-frame gate logits and the state (float32)."""
+def algorithmic_bytes(w, state_in: bool, state_out: bool, in_elem: int = 2) -> int:
+    """Bytes one gdn_forward call must move at least: q, k, v (in_elem bytes each:
+    2 for bf16, 1 for e4m3), out (bf16), the beta logits, the per-frame gate logits
+    and the state (float32)."""
     th = w.B * w.T * w.H
-    b = th * (2 * w.d_k * 2 + w.d_v * 2 + w.d_v * 2 + 4)
+    b = th * ((2 * w.d_k + w.d_v) * in_elem + w.d_v * 2 + 4)
     b += w.B * w.n_frames * w.H * 4
     st = w.B * w.H * w.d_k * w.d_v * 4
     return b + (st if state_in else 0) + (st if state_out else 0)
@@ -292,7 +296,12 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return None
     from workloads import make_inputs
-    inp = make_inputs(w)
+    if args.inputs == "fp8":
+        from oracle import gdn_reference as R
+        from workloads import make_fp8_inputs
+        inp = R.widen_fp8(make_fp8_inputs(w))           # the layer's values of the e4m3 inputs
+    else:
+        inp = make_inputs(w)
     threads = oracle_threads(w)
     budget = 150.0 / max(1, args.steps + args.warmup)      # whole run within a few minutes
     layers = calls_per_step(args, w)
@@ -377,6 +386,8 @@ def run_config(args, w):
     elif stream_step:
         api = ("gdn_state_step_ws (C ABI, device buffers, caller workspace)" if args.path == "ws"
                else "gdn_state_step (C ABI, device buffers, state in place)")
+    elif args.inputs == "fp8":
+        api = "gdn_forward_fp8 (C ABI, device buffers, no workspace)"
     else:
         api = ("gdn_forward_ws (C ABI, device buffers, caller workspace reused by every layer)"
                if args.path == "ws" else "gdn_forward (C ABI, device buffers, no workspace)")
@@ -384,7 +395,9 @@ def run_config(args, w):
                direction=("forward plus backward scan (gdn_forward_bidir)" if bidir else "forward scan"),
                gate_placement=("once per frame, at its first token (gate_mode 1)" if gate_mode
                                else "at every token of the frame"),
-               api=api)
+               api=api,
+               inputs=("q, k, v as e4m3 bytes (round to nearest even from the float32 draws), v with "
+                       "one power-of-two scale; out bf16" if args.inputs == "fp8" else "q, k, v, out bf16"))
     return cfg
 
 
@@ -536,7 +549,7 @@ def run_softmax(args, w, rank, world, local):
 # our arm
 # ----------------------------------------------------------------------------
 
-def upload_sets(w, device):
+def upload_sets(w, device, fp8=False):
     """Host (pinned later for e2e) and device copies of the workload's input sets.
 
     Returns a list of dicts with host tensors h_q, h_k, h_v, h_g, h_b, h_s (state or
@@ -548,6 +561,21 @@ def upload_sets(w, device):
     def bf16(x):
         return torch.from_numpy(bf16_bits(x).view(np.int16)).view(torch.bfloat16)
 
+    if fp8:
+        from workloads import make_fp8_inputs
+        n = BLOCK_SETS if w.name == "block" else 1
+        sets = []
+        x8s = [make_fp8_inputs(w, seed=w.seed + i) for i in range(n)]
+        for x8 in x8s:
+            h = {"h_q": torch.from_numpy(x8.q8), "h_k": torch.from_numpy(x8.k8), "h_v": torch.from_numpy(x8.v8),
+                 "h_g": torch.from_numpy(np.ascontiguousarray(x8.gate)),
+                 "h_b": torch.from_numpy(np.ascontiguousarray(x8.beta)),
+                 "h_s": None if x8.state is None else torch.from_numpy(np.ascontiguousarray(x8.state, np.float32)),
+                 "v_scale": x8.v_scale}
+            for key in ("q", "k", "v", "g", "b", "s"):
+                h[key] = None if h["h_" + key] is None else h["h_" + key].to(device)
+            sets.append(h)
+        return sets, x8s[0]
     if w.name == "sessions":
         state0, blocks = make_session_blocks(w)
         inps = blocks
@@ -577,9 +605,12 @@ def run_ours(args, w, rank, world, local):
     dist_init("nccl", world)
     layers = calls_per_step(args, w)
     lib = G.load()
-    sets, inp0 = upload_sets(w, device)
+    fp8 = args.inputs == "fp8"
+    if fp8 and (w.name == "sessions" or args.direction == "bidir" or args.gate_mode == "frame" or args.path == "ws"):
+        raise SystemExit("--inputs fp8: layer workloads (minute, clip241, block), forward scan, plain path")
+    sets, inp0 = upload_sets(w, device, fp8)
     stream_step = w.name == "sessions"
-    out = torch.empty_like(sets[0]["v"])
+    out = torch.empty(sets[0]["v"].shape, dtype=torch.bfloat16, device=device)
     st_out = torch.empty((w.B, w.H, w.d_k, w.d_v), dtype=torch.float32, device=device)
     if stream_step:
         st_out.copy_(sets[0]["s"])             # the sessions' state, carried in place
@@ -616,7 +647,11 @@ def run_ours(args, w, rank, world, local):
         else:
             s_in = x["s"].data_ptr() if (with_state_in and x["s"] is not None) else None
             args_ = (*ptr, s_in, st_out.data_ptr(), out.data_ptr())
-            if gate_mode:
+            if fp8:
+                st = lib.gdn_forward_fp8(*ptr[:3], x["v_scale"], *ptr[3:], s_in, st_out.data_ptr(),
+                                         out.data_ptr(), *dims, sptr)
+                name = "gdn_forward_fp8"
+            elif gate_mode:
                 st = lib.gdn_forward_gated(*args_, *dims, gate_mode, *ws_args, sptr)
                 name = "gdn_forward_gated"
             elif use_ws:
@@ -668,7 +703,7 @@ def run_ours(args, w, rank, world, local):
     avg_launch_s = statistics.mean(launch_ms) / 1e3
 
     peaks, peak_kind = measured_peaks()
-    abytes = algorithmic_bytes(w, state_in=with_state_in, state_out=not bidir)
+    abytes = algorithmic_bytes(w, state_in=with_state_in, state_out=not bidir, in_elem=1 if fp8 else 2)
     achieved = abytes / avg_launch_s / 1e9
     traffic, traffic_kernel = recorded_traffic()
     if bidir:
@@ -677,6 +712,8 @@ def run_ours(args, w, rank, world, local):
                   + ", combine)")
     elif use_ws:
         kernel = "gdn_ring_kernel"
+    elif fp8:
+        kernel = "gdn_seq_kernel (e4m3 inputs)"
     elif G.gdn_bf16_path(w.d_k, w.d_v, w.chunk_len) == 2:
         kernel = "gdn_seq_kernel"
     else:
@@ -697,12 +734,15 @@ def run_ours(args, w, rank, world, local):
         roofline["per_block_us"] = round(avg_launch_s * 1e6, 2)
 
     e2e = None
-    if not args.no_e2e and not bidir:
+    if not args.no_e2e and not bidir and not fp8:
         e2e = run_e2e(lib, G, w, device, stream, sets, out, st_out, world,
                       max(2, min(args.steps, 3)) if not stream_step else 1, layers if stream_step else 1, ws)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if fp8:
+            from oracle import gdn_reference as R
+            inp0 = R.widen_fp8(inp0)
         cpu = cpu_baseline(w, inp0, args.cpu_seconds, bidir=bidir)
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,

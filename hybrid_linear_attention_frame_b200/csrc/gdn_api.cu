@@ -18,7 +18,7 @@ cudaError_t ring_groups(int BH, int dv, int* groups);
 size_t ring_workspace_bytes(int G, int dv);
 cudaError_t launch_ring(const FwdParams& p, void* ws, size_t ws_bytes, cudaStream_t stream);
 bool seq_supported(int dk, int dv, int chunk_len);
-cudaError_t launch_seq(const FwdParams& p, cudaStream_t stream);
+cudaError_t launch_seq(const FwdParams& p, cudaStream_t stream, bool fp8, float v_scale);
 cudaError_t static_scratch(void** ptr, size_t* bytes);
 int read_and_clear_device_status(cudaStream_t stream);
 void set_wait_limit_ns(uint64_t ns);
@@ -89,7 +89,7 @@ int to_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; 
 
 int run_bf16(const gdn::FwdParams& p, int chunk_len, cudaStream_t stream)
 {
-    if (p.T > 0 && gdn::seq_supported(p.dk, p.dv, chunk_len)) return to_status(gdn::launch_seq(p, stream));
+    if (p.T > 0 && gdn::seq_supported(p.dk, p.dv, chunk_len)) return to_status(gdn::launch_seq(p, stream, false, 1.0f));
     if (gdn::tc_supported(p.dk, p.dv, chunk_len)) return to_status(gdn::launch_tc(p, chunk_len, stream));
     return to_status(gdn::launch_ffma<__nv_bfloat16>(p, chunk_len, stream));
 }
@@ -233,6 +233,32 @@ int gdn_forward(const void* q, const void* k, const void* v,
                       B, H, T, d_k, d_v, frame_len, chunk_len, &p);
     if (st != GDN_OK) return st;
     return run_bf16(p, chunk_len, stream);
+}
+
+int gdn_forward_fp8(const void* q8, const void* k8, const void* v8, float v_scale,
+                    const float* gate_logit, const float* beta_logit,
+                    const float* state_in, float* state_out, void* out,
+                    int B, int H, int T, int d_k, int d_v,
+                    int frame_len, int chunk_len, cudaStream_t stream)
+{
+    if (!(v_scale >= 0.0f && v_scale <= 3.4028235e38f)) return GDN_ERR_INVALID_ARG;   // NaN fails too
+    gdn::FwdParams p;
+    int st = validate(q8, k8, v8, gate_logit, beta_logit, state_in, state_out, out, true, 1,
+                      B, H, T, d_k, d_v, frame_len, chunk_len, &p);
+    if (st != GDN_OK) return st;
+    if (!gdn::seq_supported(d_k, d_v, chunk_len)) return GDN_ERR_UNSUPPORTED;
+    // out is bf16 (2 bytes per element, the inputs 1): check it at its own size
+    const int64_t F = ((int64_t)T + frame_len - 1) / frame_len;
+    const size_t nq = (size_t)B * T * H * d_k, nv = (size_t)B * T * H * d_v, no = 2 * nv;
+    const size_t ng = (size_t)B * F * H * sizeof(float), nb = (size_t)B * T * H * sizeof(float);
+    const size_t ns = (size_t)B * H * d_k * d_v * sizeof(float);
+    if (overlaps(out, no, q8, nq) || overlaps(out, no, k8, nq) || overlaps(out, no, v8, nv) ||
+        overlaps(out, no, gate_logit, ng) || overlaps(out, no, beta_logit, nb) ||
+        overlaps(out, no, state_in, ns) || overlaps(out, no, state_out, ns))
+        return GDN_ERR_INVALID_ARG;
+    // no token to read: the state passes through (the element type of q, k, v does not matter)
+    if (T == 0) return run_bf16(p, chunk_len, stream);
+    return to_status(gdn::launch_seq(p, stream, true, v_scale));
 }
 
 int gdn_state_step(const void* q, const void* k, const void* v,

@@ -74,6 +74,11 @@ constexpr uint32_t kColSacc = 384;           // state: d_k lanes x d_v columns
 // 64 x 64 token tiles use the 128-byte swizzle.
 constexpr uint32_t kAtomKQW = 6144;          // per d_k atom: K rows | Q rows | W rows (64 each)
 constexpr uint32_t kAtQ = 2048, kAtW = 4096;
+// e4m3 inputs: the k and q rows of an atom (16 bytes each, 64 rows each, so [K;Q] is
+// one 128-row K-major operand without swizzle) land in the atom's W slot, which is
+// free until the chunk's W is written; the Gram reads them there and they are
+// widened to the bf16 K and Q atoms beside it
+constexpr uint32_t kAtK8 = kAtW, kAtQ8 = kAtW + 1024;
 constexpr uint32_t kStageSc = kMaxAtoms * kAtomKQW;          // chain scalars of the stage
 constexpr uint32_t kStageBytes = kStageSc + 2048;
 constexpr uint32_t kOffV = 2 * kStageBytes;                  // v tile, d_v atoms of 64 rows
@@ -114,7 +119,8 @@ enum : uint32_t {
     B_OFREE = 21,     // output staging (the E tile) read by its TMA store
     B_OREADY = 22,    // the four output warps' rows staged
     B_WREADY = 23,    // -W written beside Q and EQS lanes 0-63 cleared (four chain warps)
-    kNumBars = 24,
+    B_KQ16 = 24,      // [2] e4m3 inputs: K and Q of a stage widened to bf16
+    kNumBars = 26,
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
@@ -148,6 +154,8 @@ static_assert(kOffS % 256 == 0 && kOffEp % 256 == 0 && kOffE % 256 == 0 && kOffV
 static_assert(kOffAXI % 16 == 0 && kOffSc % 16 == 0 && kOffMS % 16 == 0 && kOffBar % 8 == 0, "alignment");
 
 constexpr uint32_t kIdGram = idesc_bf16(128, 128, false, false);
+// kind::f8f6f4 with e4m3 A and B (format code 0 in both fields), fp32 D, both K-major
+constexpr uint32_t kIdGram8 = (1u << 4) | ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 
 __host__ __device__ constexpr uint32_t bar_count(uint32_t i) {
     return (i == B_SREADY || i == B_PEGO) ? 8u
@@ -168,6 +176,49 @@ __device__ __forceinline__ uint32_t tlane(uint32_t tmem, int quarter) {
 // Shared address of the 8 columns [c8, c8 + 8) of row r in a tile of SW32 atoms `lbo` bytes apart.
 __device__ __forceinline__ uint32_t sw32_at(uint32_t tile, uint32_t lbo, uint32_t r, uint32_t c8) {
     return tile + (c8 >> 4) * lbo + sw32_chunk_offset(r, (c8 >> 3) & 1u);
+}
+
+// ---------------------------------------------------------------- e4m3 inputs
+// Every e4m3 value, subnormals included, is a bf16 value, so the widening is exact.
+// Two e4m3 values (the low byte is the first) -> a bf16 pair (the first in the low half).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t pair) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)(pair & 0xFFFFu)));
+    float lo, hi;
+    asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"((unsigned short)(h2 & 0xFFFFu)));
+    asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"((unsigned short)(h2 >> 16)));
+    return pack_bf16x2(lo, hi);
+}
+
+// 16 e4m3 values (byte j = element j) -> one 16-column bf16 atom row (32 bytes) at
+// `row` of the 32-byte-swizzled atom `atom`
+__device__ __forceinline__ void widen16_to_atom_row(uint32_t atom, uint32_t row, const uint4& x) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        o[2 * i] = e4m3x2_to_bf16x2(w[i]);
+        o[2 * i + 1] = e4m3x2_to_bf16x2(w[i] >> 16);
+    }
+    st_shared_v4(atom + sw32_chunk_offset(row, 0), o[0], o[1], o[2], o[3]);
+    st_shared_v4(atom + sw32_chunk_offset(row, 1), o[4], o[5], o[6], o[7]);
+}
+
+// One tcgen05 MMA of kind::f8f6f4 (both operands e4m3, K = 32 per instruction).
+__device__ __forceinline__ void mma_e4m3_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p, e;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+    return r;
 }
 
 __device__ __forceinline__ void st_bf16x8(uint32_t addr, const float* x) {
@@ -232,6 +283,7 @@ __device__ __forceinline__ bool group_all(uint32_t id, uint32_t n, bool v) {
 struct SeqArgs {
     FwdParams p;
     uint64_t wait_limit_ns;
+    float v_scale;    // e4m3 inputs: v = v_scale * decode(v8) (1 for bf16 inputs)
     int G;            // CTAs
     int grid_sync;    // state_in aliases state_out: every read of it precedes every write
 };
@@ -326,6 +378,8 @@ __device__ __forceinline__ float chunk_decay(const FwdParams& p, int b, int h, i
 
 // ---------------------------------------------------------------- the kernel
 
+// kF8: q, k, v given as e4m3 bytes (v scaled by a.v_scale), widened to bf16 on the way in.
+template <bool kF8>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const SeqArgs a)
@@ -450,13 +504,25 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                                        abort_flag, lim, 21));
                 if (!ok) break;
             }
+            const uint32_t st = base + (uint32_t)s * kStageBytes;
             if (lane == 0) {
-                const uint32_t st = base + (uint32_t)s * kStageBytes, fb = bar(B_FULL + s);
-                mbar_arrive_expect_tx(fb, (uint32_t)nak * 2u * 2048u);
-                for (int at = 0; at < nak; ++at) {
-                    tma_load_4d(st + (uint32_t)at * kAtomKQW, &tm_k, fb, 16 * at, cu.pc.h, cu.c * kC, cu.pc.b);
-                    tma_load_4d(st + (uint32_t)at * kAtomKQW + kAtQ, &tm_q, fb, 16 * at, cu.pc.h, cu.c * kC,
-                                cu.pc.b);
+                if constexpr (kF8) {
+                    const uint32_t fb = bar(B_FULL + s);
+                    mbar_arrive_expect_tx(fb, (uint32_t)nak * 2u * 1024u);
+                    for (int at = 0; at < nak; ++at) {
+                        tma_load_4d(st + (uint32_t)at * kAtomKQW + kAtK8, &tm_k, fb, 16 * at, cu.pc.h, cu.c * kC,
+                                    cu.pc.b);
+                        tma_load_4d(st + (uint32_t)at * kAtomKQW + kAtQ8, &tm_q, fb, 16 * at, cu.pc.h, cu.c * kC,
+                                    cu.pc.b);
+                    }
+                } else {
+                    const uint32_t fb = bar(B_FULL + s);
+                    mbar_arrive_expect_tx(fb, (uint32_t)nak * 2u * 2048u);
+                    for (int at = 0; at < nak; ++at) {
+                        tma_load_4d(st + (uint32_t)at * kAtomKQW, &tm_k, fb, 16 * at, cu.pc.h, cu.c * kC, cu.pc.b);
+                        tma_load_4d(st + (uint32_t)at * kAtomKQW + kAtQ, &tm_q, fb, 16 * at, cu.pc.h, cu.c * kC,
+                                    cu.pc.b);
+                    }
                 }
             }
             // G (warp scan of the log-gates), beta and e^{G_L} into the stage
@@ -475,14 +541,15 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 cs[CS_BETA + i0] = (i0 < L) ? sigmoid_fast(r0) : 0.0f;
                 cs[CS_BETA + i0 + 1] = (i0 + 1 < L) ? sigmoid_fast(r1) : 0.0f;
                 if (lane == 31) cs[CS_GL] = __expf(x);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_FULL + s));
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_FULL + s));
             issued = n + 1;
         }
-        if (!ok && lane == 0)
+        if (!ok && lane == 0) {
             for (int m = max(0, issued - 2); m < issued; ++m)
                 drain_wait(bar(B_FULL + (m & 1)), (uint32_t)((m >> 1) & 1));
+        }
         __syncwarp();
     } else if (warp == kWarpGram) {
         // ======================= Gram MMAs =======================
@@ -495,13 +562,40 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
             const uint32_t st = base + (uint32_t)s * kStageBytes;
+            if constexpr (kF8) {
+                // [K;Q] in e4m3 straight from the staging: core matrices of 8 rows x 16 bytes,
+                // the next 16 bytes of K one atom further on (an odd last atom pairs with the
+                // zero tile), the next 8 rows 128 bytes on
 #pragma unroll 1
-            for (int at = 0; at < nak; ++at) {
-                const uint64_t d = dk32(st + (uint32_t)at * kAtomKQW);
-                mma_bf16_warp(tmem + kColG, d, d, kIdGram, at > 0);
+                for (int at = 0; at < nak; at += 2) {
+                    const uint32_t a0 = st + (uint32_t)at * kAtomKQW + kAtK8;
+                    const uint32_t lbo = (at + 1 < nak) ? kAtomKQW : base + kOffZ - a0;
+                    const uint64_t d = smem_desc(a0, lbo, 128, 0);
+                    mma_e4m3_warp(tmem + kColG, d, d, kIdGram8, at > 0);
+                }
+            } else {
+#pragma unroll 1
+                for (int at = 0; at < nak; ++at) {
+                    const uint64_t d = dk32(st + (uint32_t)at * kAtomKQW);
+                    mma_bf16_warp(tmem + kColG, d, d, kIdGram, at > 0);
+                }
             }
             mma_commit_warp(bar(B_G1));
             issued = n + 1;
+            if constexpr (kF8) {
+                // while the Gram reads the e4m3 rows, widen them into the stage's bf16 K and Q
+                // atoms for the W, MMA1 and MMA2 products (lanes take consecutive rows of one atom)
+#pragma unroll 4
+                for (int id = lane; id < 2 * kC * nak; id += 32) {
+                    const int isq = id >= kC * nak, rem = isq ? id - kC * nak : id;
+                    const uint32_t atom = st + (uint32_t)(rem >> 6) * kAtomKQW, r = (uint32_t)(rem & 63);
+                    const uint4 x = ld_shared_u4(atom + (isq ? kAtQ8 : kAtK8) + 16u * r);
+                    widen16_to_atom_row(atom + (isq ? kAtQ : 0u), r, x);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_KQ16 + s));
+            }
         }
         if (!ok && issued > 0 && lane == 0) drain_wait(bar(B_G1), (uint32_t)((issued - 1) & 1));
         __syncwarp();
@@ -512,13 +606,40 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         int v_issued = 0, wu_issued = 0;
         Cursor cv(a, P, warm0);
         auto load_v = [&](const Cursor& c) {
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar(B_VFULL), (uint32_t)nav * 2048u);
-                for (int at = 0; at < nav; ++at)
-                    tma_load_4d(base + kOffV + (uint32_t)at * kAtomV, &tm_v, bar(B_VFULL), 16 * at, c.pc.h, c.c * kC,
-                                c.pc.b);
+            if constexpr (kF8) {
+                // e4m3 rows straight from global memory (lanes take consecutive 16-byte
+                // pieces of a token's row), widened into the v atoms; 7 loads in flight per lane
+                const uint8_t* src = static_cast<const uint8_t*>(p.v) +
+                                     (((size_t)c.pc.b * p.T + (size_t)c.c * kC) * p.H + c.pc.h) * (size_t)dv;
+                const size_t rs = (size_t)p.H * dv;
+                const int L = c.L(), npc = kC * nav;
+                for (int b0 = 0; b0 < npc; b0 += 32 * 7) {
+                    uint4 x[7];
+#pragma unroll
+                    for (int j = 0; j < 7; ++j) {
+                        const int id = b0 + 32 * j + lane, r = id / nav, at = id - r * nav;
+                        x[j] = (id < npc && r < L)
+                                   ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * rs + 16 * at))
+                                   : make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 7; ++j) {
+                        const int id = b0 + 32 * j + lane, r = id / nav, at = id - r * nav;
+                        if (id < npc) widen16_to_atom_row(base + kOffV + (uint32_t)at * kAtomV, (uint32_t)r, x[j]);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_VFULL));
+            } else {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(B_VFULL), (uint32_t)nav * 2048u);
+                    for (int at = 0; at < nav; ++at)
+                        tma_load_4d(base + kOffV + (uint32_t)at * kAtomV, &tm_v, bar(B_VFULL), 16 * at, c.pc.h,
+                                    c.c * kC, c.pc.b);
+                }
+                __syncwarp();
             }
-            __syncwarp();
         };
         if (cv.valid()) {
             load_v(cv);
@@ -529,6 +650,7 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t eqs = tmem + kColEQS + 128u * (uint32_t)s;
             ok = mbar_wait(bar(B_TREADY), (uint32_t)(n & 1), abort_flag, lim, 24);
             ok = ok && mbar_wait(bar(B_VFULL), (uint32_t)(n & 1), abort_flag, lim, 25);
+            if constexpr (kF8) ok = ok && mbar_wait(bar(B_KQ16 + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 27);
             if (ok && n >= 2) ok = mbar_wait(bar(B_EQFREE + s), (uint32_t)(((n - 2) >> 1) & 1), abort_flag, lim, 26);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
@@ -570,6 +692,7 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ok = mbar_wait(bar(B_READY + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 31);
             ok = ok && mbar_wait(bar(B_WREADY), (uint32_t)(n & 1), abort_flag, lim, 35);
             ok = ok && mbar_wait(bar(B_SREADY), (uint32_t)(n & 1), abort_flag, lim, 32);
+            if constexpr (kF8) ok = ok && mbar_wait(bar(B_KQ16 + s), (uint32_t)((n >> 1) & 1), abort_flag, lim, 36);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
@@ -775,6 +898,7 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     for (int e = 0; e < 4; ++e) {
                         const float x = (jb + 4 * q4 + e <= i) ? xs[e] : 0.0f;
                         tv[4 * q4 + e] = x * bs[e];
+                        if constexpr (kF8) tv[4 * q4 + e] *= a.v_scale;     // U = (v_scale T) V8
                         tpv[4 * q4 + e] = x * fs[e];
                     }
                 }
@@ -984,13 +1108,30 @@ bool seq_supported(int dk, int dv, int chunk_len)
            dk <= 16 * seq::kMaxAtoms && dv <= 16 * seq::kMaxAtoms;
 }
 
-cudaError_t launch_seq(const FwdParams& p, cudaStream_t stream)
+namespace {
+// e4m3 rows of one head: 4-D view {d, H, T, B} in bytes, 16-byte x 64-token boxes
+bool make_map_u8(CUtensorMap* map, const void* base, int inner, int H, int T, int B)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)inner, (cuuint64_t)H * inner, (cuuint64_t)T * H * inner};
+    cuuint32_t box[4] = {16, 1, (cuuint32_t)seq::kC, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+cudaError_t launch_seq(const FwdParams& p, cudaStream_t stream, bool fp8, float v_scale)
 {
     if (!seq_supported(p.dk, p.dv, seq::kC) || p.T < 1) return cudaErrorInvalidValue;
+    void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, seq::SeqArgs) =
+        fp8 ? seq::gdn_seq_kernel<true> : seq::gdn_seq_kernel<false>;
     // the dynamic shared memory limit is a per-device setting of the current context: set it on
     // every call (cheap), so that every device and a context re-created after a reset get it
-    cudaError_t e = cudaFuncSetAttribute(seq::gdn_seq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)seq::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)seq::kSmemBytes);
     int dev = 0, sms = 0;
     if (e == cudaSuccess) e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1001,17 +1142,24 @@ cudaError_t launch_seq(const FwdParams& p, cudaStream_t stream)
     // 32-byte boxes, each read by exactly one CTA: no L2 promotion, so that a box
     // fetches its own sectors only and not the neighbouring heads' bytes
     const CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_NONE;
-    CUtensorMap mo;
-    if (!make_map(&mq, p.q, p.dk, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B, promo) ||
-        !make_map(&mk, p.k, p.dk, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B, promo) ||
-        !make_map(&mv, p.v, p.dv, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B, promo))
+    if (fp8) {
+        // e4m3 q and k through TMA (16-byte boxes); v is read by the v loader warp directly
+        if (!make_map_u8(&mq, p.q, p.dk, p.H, p.T, p.B) || !make_map_u8(&mk, p.k, p.dk, p.H, p.T, p.B))
+            return cudaErrorInvalidValue;
+        mv = mq;
+    } else if (!make_map(&mq, p.q, p.dk, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B, promo) ||
+               !make_map(&mk, p.k, p.dk, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B, promo) ||
+               !make_map(&mv, p.v, p.dv, p.H, p.T, p.B, 16, CU_TENSOR_MAP_SWIZZLE_32B, promo)) {
         return cudaErrorInvalidValue;
+    }
+    CUtensorMap mo;
     // output: whole 64-token rows of d_v per store (no swizzle); the q map stands in when there is no output
     if (p.out ? !make_map(&mo, p.out, p.dv, p.H, p.T, p.B, p.dv, CU_TENSOR_MAP_SWIZZLE_NONE, promo) : (mo = mq, false))
         return cudaErrorInvalidValue;
     seq::SeqArgs args;
     args.p = p;
     args.wait_limit_ns = g_wait_limit_ns;
+    args.v_scale = fp8 ? v_scale : 1.0f;
     args.G = (int)(U < sms ? U : sms);
     args.grid_sync = (p.state_in != nullptr && (const void*)p.state_in == (const void*)p.state_out) ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
@@ -1024,7 +1172,7 @@ cudaError_t launch_seq(const FwdParams& p, cudaStream_t stream)
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = args.grid_sync ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, seq::gdn_seq_kernel, mq, mk, mv, mo, args);
+    return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, args);
 }
 
 }  // namespace gdn

@@ -23,7 +23,7 @@ EXPORTS = ("gdn_forward", "gdn_state_step", "gdn_forward_f32", "gdn_state_step_f
            "gdn_forward_host", "gdn_workspace_bytes", "gdn_forward_ws", "gdn_state_step_ws",
            "gdn_forward_host_ws", "gdn_forward_static_ws", "gdn_forward_gated",
            "gdn_forward_gated_f32", "gdn_bidir_workspace_bytes", "gdn_forward_bidir",
-           "gdn_forward_bidir_f32", "gdn_softmax_attention", "gdn_set_wait_limit_ns", "gdn_status_string",
+           "gdn_forward_bidir_f32", "gdn_forward_fp8", "gdn_softmax_attention", "gdn_set_wait_limit_ns", "gdn_status_string",
            "gdn_get_last_device_status", "gdn_bf16_path", "gdn_version")
 
 
@@ -83,6 +83,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.gdn_forward_bidir.restype = I
     lib.gdn_forward_bidir_f32.argtypes = [P] * 6 + [I] * 7 + [P, Z, P]
     lib.gdn_forward_bidir_f32.restype = I
+    lib.gdn_forward_fp8.argtypes = [P] * 3 + [ctypes.c_float] + [P] * 5 + [I] * 7 + [P]
+    lib.gdn_forward_fp8.restype = I
     lib.gdn_softmax_attention.argtypes = [P] * 4 + [I] * 9 + [P]
     lib.gdn_softmax_attention.restype = I
     lib.gdn_status_string.argtypes = [I]
@@ -132,6 +134,15 @@ def gdn_forward(q, k, v, gate_logit, beta_logit, state_in, state_out, out,
                             _ptr(state_in), _ptr(state_out), _ptr(out),
                             B, H, T, d_k, d_v, frame_len, chunk_len, _stream(stream))
     return _check(st, "gdn_forward", check)
+
+
+def gdn_forward_fp8(q8, k8, v8, v_scale, gate_logit, beta_logit, state_in, state_out, out,
+                    B, H, T, d_k, d_v, frame_len, chunk_len, stream=None, check=True) -> int:
+    """q8, k8, v8: e4m3 bytes (uint8 tensors); v = v_scale * e4m3(v8); out bf16."""
+    st = load().gdn_forward_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(v_scale), _ptr(gate_logit),
+                                _ptr(beta_logit), _ptr(state_in), _ptr(state_out), _ptr(out),
+                                B, H, T, d_k, d_v, frame_len, chunk_len, _stream(stream))
+    return _check(st, "gdn_forward_fp8", check)
 
 
 def gdn_state_step(q, k, v, gate_logit, beta_logit, state, out,

@@ -128,6 +128,31 @@ int gdn_state_step_f32(const float* q, const float* k, const float* v,
                        int frame_len, int chunk_len, cudaStream_t stream);
 
 /*
+ * FP8 input variant (the pages ship fp8 precision modes for Stage-1: FlashDreams
+ * SANA-WM streaming runner page, requirements and CLI sections, precision flags;
+ * they give no scheme, so the library reads it as follows).  q8, k8, v8 hold OCP
+ * e4m3 bytes (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits,
+ * subnormals, no infinities, 0x7F / 0xFF NaN) in the layouts of gdn_forward
+ * ([B, T, H, d] row-major, one byte per element).  The layer computes
+ * gdn_forward on q = e4m3(q8), k = e4m3(k8), v = v_scale * e4m3(v8): q and k
+ * need no scale, since their L2 normalisation cancels any positive one; v_scale
+ * (finite, >= 0) is one float32 per call.  out (bf16), the logits and the state
+ * (float32) are as in gdn_forward, and state_in may alias state_out (a streaming
+ * step in place).  Every e4m3 value is exactly a bf16 value, so the kernel widens
+ * the tiles to bf16 in shared memory and the arithmetic is that of gdn_forward's
+ * sequence-parallel kernel; v_scale is applied to the bf16 T operand of U = T V.
+ * The HBM bytes per token and head drop from 900 to 564 at d = 112.
+ * Supported: d_k, d_v multiples of 16 in [16, 112], chunk_len 64 (else
+ * GDN_ERR_UNSUPPORTED); q8, k8, v8 16-byte aligned.  NaN codes give NaN
+ * outputs.  Errors otherwise as gdn_forward; nothing is enqueued on an error.
+ */
+int gdn_forward_fp8(const void* q8, const void* k8, const void* v8, float v_scale,
+                    const float* gate_logit, const float* beta_logit,
+                    const float* state_in, float* state_out, void* out,
+                    int B, int H, int T, int d_k, int d_v,
+                    int frame_len, int chunk_len, cudaStream_t stream);
+
+/*
  * End-to-end call with HOST buffers (bf16 q/k/v/out, float32 logits/state):
  * copies the inputs to the caller's device buffers d_* on `stream`, runs
  * gdn_forward, copies out (and the final state, if h_state_out is not NULL)

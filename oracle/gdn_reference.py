@@ -47,6 +47,12 @@ gate of its own frame (at every token):
 
 ``token_recurrence_backward`` is that backward loop, ``bidirectional`` the sum,
 ``c_bidirectional`` the C form of the sum.
+
+The fp8 input variant (the FlashDreams SANA-WM streaming runner page ships fp8
+precision modes without a scheme) is read as: q, k, v given as OCP e4m3 bytes,
+v with one float scale, v = v_scale * e4m3(v8); the layer is the recurrence
+above on those values.  ``decode_e4m3`` writes out the e4m3 format and
+``widen_fp8`` turns such inputs into the float64 values every form here takes.
 """
 
 import ctypes
@@ -65,6 +71,40 @@ _SRC_PATH = os.path.join(_HERE, "gdn_oracle.c")
 # ----------------------------------------------------------------------------
 # elementwise definitions
 # ----------------------------------------------------------------------------
+
+
+def decode_e4m3(codes):
+    """OCP e4m3 bytes -> float64: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+    bits; exponent field 0 holds the subnormals m/8 * 2^-6, field 1..15 the normals
+    (1 + m/8) * 2^(e-7); the one code with all of exponent and mantissa set
+    (0x7F, 0xFF) is NaN and there are no infinities, so the largest value is 448."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 0xF) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+class Widened:
+    """fp8 inputs as the float64 values of the layer (the fields the forms here read)."""
+
+    def __init__(self, x8):
+        self.q = decode_e4m3(x8.q8)
+        self.k = decode_e4m3(x8.k8)
+        self.v = float(x8.v_scale) * decode_e4m3(x8.v8)
+        self.gate = x8.gate
+        self.beta = x8.beta
+        self.state = x8.state
+        self.frame_len = x8.frame_len
+        self.gate_mode = getattr(x8, "gate_mode", GATE_EVERY_TOKEN)
+        self.io_dtype = "f32"
+
+
+def widen_fp8(x8):
+    """q = e4m3(q8), k = e4m3(k8), v = v_scale * e4m3(v8), the rest unchanged."""
+    return Widened(x8)
 
 def softplus(x):
     """log(1 + e^x), computed without overflow."""

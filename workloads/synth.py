@@ -120,3 +120,70 @@ def make_session_blocks(w: Workload, n_blocks: Optional[int] = None):
             beta=np.concatenate([p.beta for p in parts]), state=None,
             io_dtype=w.io_dtype, frame_len=w.frame_len))
     return state0, blocks
+
+
+# ---------------------------------------------------------------- e4m3 inputs
+#
+# The fp8 input variant takes q, k and v as OCP e4m3 bytes.  Producing those bytes
+# is the caller's quantisation, not part of the layer, so it lives here with the
+# other input generation: round-to-nearest-even from the float32 draws, saturating
+# at +-448 (the largest finite e4m3 value).  q and k are encoded as drawn; v is
+# divided by one power-of-two scale first, so that max |v| / scale <= 448 and the
+# scaled values stay exactly representable in float32.
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """float32 -> e4m3 codes (uint8): nearest value, ties to even, saturating."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    neg = np.signbit(x)
+    m = np.minimum(np.abs(x), 448.0)
+    # exponent of the binade (subnormals share the quantum of the lowest binade)
+    e = np.clip(np.floor(np.log2(np.maximum(m, 2.0 ** -10))), -6, 8)
+    quantum = np.exp2(e - 3)
+    qv = np.minimum(np.round(m / quantum) * quantum, 448.0)     # np.round: ties to even
+    sub = qv < 2.0 ** -6
+    e2 = np.floor(np.log2(np.where(sub, 1.0, qv)))
+    mant = np.where(sub, qv * 512.0, (qv / np.exp2(e2) - 1.0) * 8.0)
+    expo = np.where(sub, 0.0, e2 + 7.0)
+    code = (expo.astype(np.int64) << 3) | mant.astype(np.int64)
+    return (code | (neg.astype(np.int64) << 7)).astype(np.uint8)
+
+
+def v_scale_for(v: np.ndarray) -> float:
+    """The power-of-two scale that maps max |v| into the e4m3 range."""
+    amax = float(np.max(np.abs(v))) if v.size else 0.0
+    if amax == 0.0:
+        return 1.0
+    return float(2.0 ** np.ceil(np.log2(amax / 448.0)))
+
+
+@dataclass
+class Fp8Inputs:
+    q8: np.ndarray          # uint8 e4m3 codes [B, T, H, d_k]
+    k8: np.ndarray          # uint8 e4m3 codes [B, T, H, d_k]
+    v8: np.ndarray          # uint8 e4m3 codes [B, T, H, d_v]
+    v_scale: float          # v = v_scale * e4m3(v8)
+    gate: np.ndarray
+    beta: np.ndarray
+    state: Optional[np.ndarray]
+    frame_len: int
+    gate_mode: int = 0
+
+
+def to_fp8(inp: Inputs, v_scale: Optional[float] = None) -> Fp8Inputs:
+    """Encode float32 draws (io_dtype 'f32') as e4m3 inputs."""
+    if inp.io_dtype != "f32":
+        raise ValueError("encode the float32 draws, not rounded copies")
+    s = v_scale_for(inp.v) if v_scale is None else float(v_scale)
+    v = (inp.v.astype(np.float64) / s).astype(np.float32)
+    return Fp8Inputs(e4m3_encode(inp.q), e4m3_encode(inp.k), e4m3_encode(v), s,
+                     inp.gate, inp.beta, inp.state, inp.frame_len, inp.gate_mode)
+
+
+def make_fp8_inputs(w: Workload, T: Optional[int] = None, seed: Optional[int] = None) -> Fp8Inputs:
+    """e4m3 inputs of one call of workload ``w``: the same draws as ``make_inputs``
+    (before bf16 rounding), encoded."""
+    rng = np.random.Generator(np.random.PCG64(w.seed if seed is None else seed))
+    inp = draw(rng, w.B, w.H, w.T if T is None else T, w.d_k, w.d_v, w.frame_len,
+               "f32", w.gate_mean, w.gate_std, w.beta_mean, w.beta_std, w.state_std)
+    return to_fp8(inp)
