@@ -97,7 +97,8 @@ constexpr uint32_t kOffAXI = kOffE + kMaxAtoms * kAtomE;     // fp32 [64][kXS]: 
 constexpr uint32_t kScFloats = 13 * 64 + 16;
 constexpr uint32_t kOffSc = kOffAXI + 64 * kXS * 4;          // prep scalar table
 constexpr uint32_t kOffMS = kOffSc + kScFloats * 4;         // the UT inverse's scratch
-constexpr uint32_t kMSBytes = 4 * tc::kMS * 32 * 4;
+constexpr int kCS = 36;                                      // row stride (floats) of its level-2 product
+constexpr uint32_t kMSBytes = 32 * kCS * 4;
 constexpr uint32_t kOffBar = kOffMS + kMSBytes;
 enum : uint32_t {
     B_FULL = 0,       // [2] q/k tiles of a stage landed and its gates written
@@ -152,6 +153,7 @@ static_assert(kOffS % 256 == 0 && kOffEp % 256 == 0 && kOffE % 256 == 0 && kOffV
                   kAtomKQW % 256 == 0 && kAtomS % 256 == 0,
               "SW32 alignment");
 static_assert(kOffAXI % 16 == 0 && kOffSc % 16 == 0 && kOffMS % 16 == 0 && kOffBar % 8 == 0, "alignment");
+static_assert(4 * tc::kMS * 32 * 4 <= kMSBytes, "level-1 scratch fits");
 
 constexpr uint32_t kIdGram = idesc_bf16(128, 128, false, false);
 // kind::f8f6f4 with e4m3 A and B (format code 0 in both fields), fp32 D, both K-major
@@ -377,6 +379,93 @@ __device__ __forceinline__ float chunk_decay(const FwdParams& p, int b, int h, i
 }
 
 // ---------------------------------------------------------------- the kernel
+
+// ---------------------------------------------------------------- UT inverse
+// (I + A)^{-1} for the 64 x 64 unit lower-triangular I + A (A strictly lower, stored
+// transposed above the diagonal of AXI) into the lower triangle of AXI, by block
+// combination: [[X, 0], [C, Y]]^{-1} = [[X^-1, 0], [-Y^-1 C X^-1, Y^-1]].
+//
+// Diagonal 16 x 16 blocks and the first level (16 -> 32) on the four A warps (128
+// threads, `st`): forward substitution in fp32, one column per thread, the column of A
+// that a step needs read as four 16-byte vectors (it is a row of the transposed
+// storage); then the two 16 x 16 combinations on mma.sync tf32, one 8-column tile per
+// warp, as in tc::unit_lower_inverse_64.
+__device__ __forceinline__ void inverse_levels01(float* AXI, float* MS, int st) {
+    using tc::AAt;
+    using tc::XIv;
+    const int pw = st >> 5, lane = st & 31, g = lane >> 2, t = lane & 3;
+    if (st < 64) {
+        const int o = 16 * (st >> 4), j = st & 15;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = (i == j) ? 1.0f : 0.0f;
+#pragma unroll
+        for (int m = 0; m < 15; ++m) {
+            const float* arow = AXI + (o + m) * kXS + o;     // A(o + i, o + m) at column o + i
+            float a[16];
+#pragma unroll
+            for (int q4 = (m + 1) / 4; q4 < 4; ++q4) {
+                const float4 v = *reinterpret_cast<const float4*>(arow + 4 * q4);
+                a[4 * q4] = v.x; a[4 * q4 + 1] = v.y; a[4 * q4 + 2] = v.z; a[4 * q4 + 3] = v.w;
+            }
+#pragma unroll
+            for (int i = m + 1; i < 16; ++i) x[i] = fmaf(-a[i], x[m], x[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (i >= j) AXI[(o + i) * kXS + o + j] = x[i];
+    }
+    named_bar_sync(tc::kBarSolve, 128);
+    // blocks (1,0) and (3,2): Y = -D_hi^{-1} (A_{hi,lo} D_lo^{-1}); warp -> (pair, 8 columns)
+    float* MSw = MS + pw * 32 * tc::kMS;
+    const int pr = pw >> 1, n0 = 8 * (pw & 1);
+    const int hi = 16 * (2 * pr + 1), lo = 16 * (2 * pr);
+    float m1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    tc::tile16x8<16>(m1, [&](int r, int k) { return AAt(AXI, hi + r, lo + k); },
+                     [&](int k, int n) { return XIv(AXI, lo + k, lo + n0 + n); }, lane);
+    MSw[g * tc::kMS + 2 * t] = m1[0];
+    MSw[g * tc::kMS + 2 * t + 1] = m1[1];
+    MSw[(g + 8) * tc::kMS + 2 * t] = m1[2];
+    MSw[(g + 8) * tc::kMS + 2 * t + 1] = m1[3];
+    __syncwarp();
+    float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    tc::tile16x8<16>(y, [&](int r, int k) { return XIv(AXI, hi + r, hi + k); },
+                     [&](int k, int n) { return MSw[k * tc::kMS + n]; }, lane);
+    AXI[(hi + g) * kXS + lo + n0 + 2 * t] = -y[0];
+    AXI[(hi + g) * kXS + lo + n0 + 2 * t + 1] = -y[1];
+    AXI[(hi + g + 8) * kXS + lo + n0 + 2 * t] = -y[2];
+    AXI[(hi + g + 8) * kXS + lo + n0 + 2 * t + 1] = -y[3];
+}
+
+// The second level (32 -> 64) on all eight prep warps (`w` = 0..7): C = A_21 X_11
+// (one 16 x 8 tile each), then X_21 = -X_22 C (X_22 lower triangular, so the upper
+// row tile needs only the first 16 columns of it).  The caller's barrier over the
+// eight warps precedes it (levels 0-1 done) and follows it.
+__device__ __forceinline__ void inverse_level2(float* AXI, float* C, int w, int lane, uint32_t bar_id) {
+    using tc::AAt;
+    using tc::XIv;
+    const int g = lane >> 2, t = lane & 3, mt = w >> 2, c0 = 8 * (w & 3);
+    float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    tc::tile16x8<32>(c, [&](int r, int k) { return AAt(AXI, 32 + 16 * mt + r, k); },
+                     [&](int k, int n) { return XIv(AXI, k, c0 + n); }, lane);
+    C[(16 * mt + g) * kCS + c0 + 2 * t] = c[0];
+    C[(16 * mt + g) * kCS + c0 + 2 * t + 1] = c[1];
+    C[(16 * mt + g + 8) * kCS + c0 + 2 * t] = c[2];
+    C[(16 * mt + g + 8) * kCS + c0 + 2 * t + 1] = c[3];
+    named_bar_sync(bar_id, kPrepThreads);
+    float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (mt == 0)
+        tc::tile16x8<16>(y, [&](int r, int k) { return XIv(AXI, 32 + r, 32 + k); },
+                         [&](int k, int n) { return C[k * kCS + c0 + n]; }, lane);
+    else
+        tc::tile16x8<32>(y, [&](int r, int k) { return XIv(AXI, 48 + r, 32 + k); },
+                         [&](int k, int n) { return C[k * kCS + c0 + n]; }, lane);
+    const int r0 = 32 + 16 * mt + g;
+    AXI[r0 * kXS + c0 + 2 * t] = -y[0];
+    AXI[r0 * kXS + c0 + 2 * t + 1] = -y[1];
+    AXI[(r0 + 8) * kXS + c0 + 2 * t] = -y[2];
+    AXI[(r0 + 8) * kXS + c0 + 2 * t + 1] = -y[3];
+}
 
 // kF8: q, k, v given as e4m3 bytes (v scaled by a.v_scale), widened to bf16 on the way in.
 template <bool kF8>
@@ -874,11 +963,13 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (qtr < 2) {
                 named_bar_sync(kBarA, 128);      // A complete
                 if (pw == 0 && lane == 0) mbar_arrive(bar(B_GFREE));
-                tc::unit_lower_inverse_64(AXI, MSf, 32 * ((pw & 1) | ((pw >> 2) << 1)) + lane);
+                inverse_levels01(AXI, MSf, 32 * ((pw & 1) | ((pw >> 2) << 1)) + lane);
             } else {
                 named_bar_sync(kBarP, 128);      // P complete
                 if (pw == 2 && lane == 0) mbar_arrive(bar(B_GFREE));
             }
+            named_bar_sync(kBarPrep, kPrepThreads);
+            inverse_level2(AXI, MSf, pw, lane, kBarPrep);
             bool okw = true;
             if (n > 0) okw = mbar_wait(bar(B_WU + (uint32_t)((n - 1) & 1)), (uint32_t)(((n - 1) >> 1) & 1), abort_flag, lim, 42);
             if (!group_all(kBarPrep, kPrepThreads, okw)) return false;
