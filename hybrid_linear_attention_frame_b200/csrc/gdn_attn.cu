@@ -21,7 +21,9 @@
 //   P in bf16 to shared memory, O += P V on the tensor cores into TMEM.
 // K tiles are triple-buffered and V tiles double-buffered, loaded by TMA (128-byte
 // swizzle, rows past the end of the sequence read as zeros and are masked).
-// Warp 0 issues the copies and the MMAs.  Every wait is bounded.
+// Warp 8 issues the copies and the MMAs; warps 0-7 only run the softmax, and the two
+// sides meet at mbarriers: S ready / S read, P written / P V done.  Every wait is
+// bounded.
 #include "gdn_common.cuh"
 #include "gdn_sm100.cuh"
 
@@ -30,7 +32,9 @@ namespace attn {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;                  // two threads per query row
+constexpr int kSoftThreads = 256;              // softmax warps 0-7: two threads per query row
+constexpr int kProducerWarp = 8;               // copies and MMAs
+constexpr int kThreads = kSoftThreads + 32;
 constexpr int kHalfKeys = 64;                  // keys of a tile per thread
 constexpr int kBM = 128;                       // queries per CTA
 constexpr int kBN = 128;                       // keys per tile
@@ -43,11 +47,16 @@ constexpr uint32_t kOffV = kOffK + kKStages * kOp;
 constexpr uint32_t kOffP = kOffV + kVStages * kOp;
 constexpr uint32_t kOffBar = kOffP + kOp;
 enum : uint32_t { kBarQ = 0, kBarK = 1, kBarV = kBarK + kKStages, kBarS = kBarV + kVStages, kBarPV = kBarS + 2,
-                  kNumBars = kBarPV + 1 };
+                  kBarSFree = kBarPV + 1,   // [2] the softmax warps have read a score buffer (8 arrivals)
+                  kBarPFull = kBarSFree + 2, // P written and O rescaled (8 arrivals)
+                  kNumBars = kBarPFull + 1 };
+__host__ __device__ constexpr uint32_t bar_count(uint32_t i) {
+    return (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull) ? 8u : 1u;
+}
 constexpr uint32_t kOffAbort = kOffBar + 8u * kNumBars;
 constexpr uint32_t kOffTmemSlot = kOffAbort + 8u;
 constexpr uint32_t kOffX = kOffTmemSlot + 16u;                 // 256 floats: the two halves' exchange
-constexpr uint32_t kSmemBytes = kOffX + 4u * kThreads + 1024u; // + slack for 1024-byte alignment
+constexpr uint32_t kSmemBytes = kOffX + 4u * kSoftThreads + 1024u; // + slack for 1024-byte alignment
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "SW128 tiles need 1024-B alignment");
 
@@ -55,7 +64,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;                  // two 128-column score buffers
 constexpr uint32_t kColO = 256;                // the d_v-column output accumulator
 constexpr float kMoveRef = 8.0f;               // log2 units: p stays below 2^8
-constexpr uint32_t kBarGroup = 1;              // named barrier of all the CTA's threads
+constexpr uint32_t kBarGroup = 1;              // named barrier of the softmax warps
 
 constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);
 
@@ -150,7 +159,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto tile_start = [&](int j) { return j < nA ? kBN * j : startB + kBN * (j - nA); };
 
     // ---- this thread's query row, half of the keys and its row's key set ----
-    const int row = tid & (kBM - 1), half = tid / kBM;
+    const int row = tid & (kBM - 1), half = (tid / kBM) & 1;      // (softmax threads)
     const int t = t0 + row;
     const int te = min(t, T - 1);
     const int ws = max(0, te / bl - a.cached) * bl;
@@ -161,7 +170,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tmem_relinquish();
     }
     if (tid == 32) {
-        for (uint32_t i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+        for (uint32_t i = 0; i < kNumBars; ++i) mbar_init(bar(i), bar_count(i));
         fence_mbar_init();
         *abort_flag = 0;
         tma_prefetch_desc(&tm_q);
@@ -178,44 +187,43 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t idpv = idesc_bf16(128, a.dv, false, true);
     const int nks = a.dk / 16;
 
-    // issue / wait bookkeeping (warp 0 issues; counts are uniform within a warp)
-    int k_issued = 0, k_waited = 0, v_issued = 0, v_waited = 0, s_issued = 0, pv_issued = 0;
-    int s_waited = 0, pv_waited = 0;
-    bool q_pending = false;
-    auto load_k = [&](int j) {
-        if (lane == 0) {
-            const uint32_t b = bar(kBarK + j % kKStages), dst = base + kOffK + (uint32_t)(j % kKStages) * kOp;
-            mbar_arrive_expect_tx(b, kOp);
-            tma_load_4d(dst, &tm_k, b, 0, h, tile_start(j), bb);
-            tma_load_4d(dst + kBox, &tm_k, b, 64, h, tile_start(j), bb);
-        }
-        __syncwarp();
-        k_issued = j + 1;
-    };
-    auto load_v = [&](int j) {
-        if (lane == 0) {
-            const uint32_t b = bar(kBarV + j % kVStages), dst = base + kOffV + (uint32_t)(j % kVStages) * kOp;
-            mbar_arrive_expect_tx(b, kOp);
-            tma_load_4d(dst, &tm_v, b, 0, h, tile_start(j), bb);
-            tma_load_4d(dst + kBox, &tm_v, b, 64, h, tile_start(j), bb);
-        }
-        __syncwarp();
-        v_issued = j + 1;
-    };
-    // S of tile j into score buffer j & 1, once its K tile has landed (warp 0)
-    auto start_s = [&](int j) -> bool {
-        const bool got = mbar_wait(bar(kBarK + j % kKStages), (uint32_t)((j / kKStages) & 1), abort_flag, lim, 21);
-        if (!__all_sync(0xffffffffu, got)) return false;      // the MMA issue below is warp-collective
-        k_waited = j + 1;
-        tc_fence_after();
-        issue_s(base + kOffQ, base + kOffK + (uint32_t)(j % kKStages) * kOp, tmem + kColS + 128u * (j & 1), nks);
-        mma_commit_warp(bar(kBarS + (j & 1)));
-        s_issued = j + 1;
-        return true;
-    };
-
-    bool ok = true;
-    if (warp == 0) {
+    if (warp == kProducerWarp) {
+        // ======================= copies and MMAs =======================
+        // issued / waited counts (uniform within the warp) for the drain on the way out
+        int k_issued = 0, k_waited = 0, v_issued = 0, v_waited = 0, s_issued = 0, s_waited = 0;
+        int pv_issued = 0, pv_waited = 0;
+        bool q_pending = false, ok = true;
+        auto load_k = [&](int j) {
+            if (lane == 0) {
+                const uint32_t b = bar(kBarK + j % kKStages), dst = base + kOffK + (uint32_t)(j % kKStages) * kOp;
+                mbar_arrive_expect_tx(b, kOp);
+                tma_load_4d(dst, &tm_k, b, 0, h, tile_start(j), bb);
+                tma_load_4d(dst + kBox, &tm_k, b, 64, h, tile_start(j), bb);
+            }
+            __syncwarp();
+            k_issued = j + 1;
+        };
+        auto load_v = [&](int j) {
+            if (lane == 0) {
+                const uint32_t b = bar(kBarV + j % kVStages), dst = base + kOffV + (uint32_t)(j % kVStages) * kOp;
+                mbar_arrive_expect_tx(b, kOp);
+                tma_load_4d(dst, &tm_v, b, 0, h, tile_start(j), bb);
+                tma_load_4d(dst + kBox, &tm_v, b, 64, h, tile_start(j), bb);
+            }
+            __syncwarp();
+            v_issued = j + 1;
+        };
+        // S of tile j into score buffer j & 1, once its K tile has landed
+        auto start_s = [&](int j) -> bool {
+            const bool got = mbar_wait(bar(kBarK + j % kKStages), (uint32_t)((j / kKStages) & 1), abort_flag, lim, 21);
+            if (!__all_sync(0xffffffffu, got)) return false;      // the MMA issue below is warp-collective
+            k_waited = j + 1;
+            tc_fence_after();
+            issue_s(base + kOffQ, base + kOffK + (uint32_t)(j % kKStages) * kOp, tmem + kColS + 128u * (j & 1), nks);
+            mma_commit_warp(bar(kBarS + (j & 1)));
+            s_issued = j + 1;
+            return true;
+        };
         if (lane == 0) {
             mbar_arrive_expect_tx(bar(kBarQ), kOp);
             tma_load_4d(base + kOffQ, &tm_q, bar(kBarQ), 0, h, t0, bb);
@@ -223,164 +231,184 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         __syncwarp();
         q_pending = true;
-        load_k(0);
-        if (n > 1) load_k(1);
-        load_v(0);
+        for (int j = 0; j < min(n, kKStages); ++j) load_k(j);
+        for (int j = 0; j < min(n, kVStages); ++j) load_v(j);
         ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarQ), 0, abort_flag, lim, 20));
         if (ok) q_pending = false;
         ok = ok && start_s(0);
-    }
-
-    // `ok` is this thread's own record (a failed wait of warp 0 stays private until the
-    // next vote); `alive` is what every thread agreed on at the last vote.  Threads
-    // leave the loop only together, after a vote, so no barrier is left half-arrived.
-    bool alive = true;
-    float m_ref = -INFINITY, l = 0.0f;
-    for (int j = 0; j < n; ++j) {
-        // ---- warp 0: next tile's S, and the K tile after it ----
-        if (warp == 0 && ok) {
-            if (j + 1 < n) ok = start_s(j + 1);
-            if (ok && j + 2 < n) load_k(j + 2);
-        }
-        // ---- this tile's scores ----
-        ok = ok && mbar_wait(bar(kBarS + (j & 1)), (uint32_t)((j >> 1) & 1), abort_flag, lim, 22);
-        if (!group_all(kBarGroup, kThreads, ok)) { alive = false; break; }
-        s_waited = j + 1;
-        tc_fence_after();
-        const int s0 = tile_start(j) + kHalfKeys * half;     // this thread's first key
-        const bool sink_tile = j < nA;
-        float x[kHalfKeys];
-#pragma unroll
-        for (int c = 0; c < kHalfKeys / 16; ++c)
-            tmem_ld16(lane_base + kColS + 128u * (j & 1) + (uint32_t)(kHalfKeys * half) + 16u * c,
-                      *reinterpret_cast<float(*)[16]>(&x[16 * c]));
-        // Are all of this thread's keys inside its row's key set?  (Then no per-key mask.)
-        bool full;
-        if (sink_tile) full = s0 + kHalfKeys <= sink;
-        else if (split) full = s0 >= ws && s0 + kHalfKeys <= we;
-        else full = (ws <= sink) ? (s0 + kHalfKeys <= max(sink, we))
-                                 : (s0 + kHalfKeys <= sink || (s0 >= ws && s0 + kHalfKeys <= we));
-        tmem_wait_ld();
-        if (!full) {
-#pragma unroll
-            for (int i = 0; i < kHalfKeys; ++i) {
-                const int s = s0 + i;
-                const bool valid = sink_tile ? (s < sink)
-                                             : (s < T && ((!split && s < sink) || (s >= ws && s < we)));
-                x[i] = valid ? x[i] : -INFINITY;
+        for (int j = 0; ok && j < n; ++j) {
+            // the next tile's S, once the softmax has read the buffer it goes into (tile j - 1's)
+            if (j + 1 < n) {
+                if (j >= 1)
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarSFree + ((j + 1) & 1)), (uint32_t)(((j - 1) >> 1) & 1),
+                                                           abort_flag, lim, 26));
+                ok = ok && start_s(j + 1);
             }
-        }
-        // maximum of the raw scores (the scale is positive) over both halves of the row
-        float mx[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) mx[e] = x[e];
-#pragma unroll
-        for (int i = 4; i < kHalfKeys; ++i) mx[i & 3] = fmaxf(mx[i & 3], x[i]);
-        xchg[tid] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        named_bar_sync(kBarGroup, kThreads);
-        const float mt = fmaxf(xchg[tid], xchg[tid ^ kBM]) * a.scale_log2;
-        const bool move = mt > m_ref + kMoveRef;   // the same decision in both threads of the row
-        float alpha = 1.0f;
-        if (move) {
-            alpha = ex2(m_ref - mt);
-            m_ref = mt;
-        }
-        const float neg_mr = (m_ref == -INFINITY) ? 0.0f : -m_ref;
-        float sm[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[kHalfKeys / 2];
-#pragma unroll
-        for (int i = 0; i < kHalfKeys / 2; ++i) {
-            const float p0 = ex2(fmaf(x[2 * i], a.scale_log2, neg_mr));
-            const float p1 = ex2(fmaf(x[2 * i + 1], a.scale_log2, neg_mr));
-            sm[i & 3] += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
-        }
-        const float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);     // this half's part of the row sum
-        l = l * alpha + sum;
-        // ---- the previous P V must be done: P's buffer is reused and O may be rescaled ----
-        if (j > 0) {
-            ok = mbar_wait(bar(kBarPV), (uint32_t)((j - 1) & 1), abort_flag, lim, 23);
-            if (!group_all(kBarGroup, kThreads, ok)) { alive = false; break; }
-            pv_waited = j;
-            tc_fence_after();
-        }
-        if (warp == 0 && j + 1 < n) load_v(j + 1);
-        // TMEM loads and stores are warp-collective: the whole warp rescales when any
-        // of its rows moved its reference (the others with alpha = 1)
-        if (__any_sync(0xffffffffu, move && j > 0)) {
-            const float f = (move && j > 0) ? alpha : 1.0f;
-#pragma unroll 1
-            for (int c = c_lo; c < c_hi; ++c) {
-                float o[16];
-                tmem_ld16(lane_base + kColO + 16u * c, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) o[e] *= f;
-                tmem_st16(lane_base + kColO + 16u * c, o);
+            // tile j's K slot takes tile j + 3 once S(j) is done
+            if (ok && j + kKStages < n) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarS + (j & 1)), (uint32_t)((j >> 1) & 1), abort_flag, lim, 27));
+                if (ok) {
+                    s_waited = j + 1;
+                    load_k(j + kKStages);
+                }
             }
-            tmem_wait_st();
-        }
-        // ---- this thread's 64 keys of the P row (bf16) into its box of the K-major SW128 operand ----
-        {
-            const uint32_t prow = base + kOffP + (uint32_t)half * kBox + (uint32_t)row * 128u;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_shared_v4(prow + ((uint32_t)(c ^ (row & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                             pk[4 * c + 3]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        named_bar_sync(kBarGroup, kThreads);
-        if (warp == 0) {
-            tc_fence_after();
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(bar(kBarV + j % kVStages), (uint32_t)((j / kVStages) & 1), abort_flag, lim, 24));
+            // V slot of tile j - 1 takes tile j + 1 once P V(j - 1) is done
+            if (ok && j >= 1 && j + 1 < n) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarPV), (uint32_t)((j - 1) & 1), abort_flag, lim, 28));
+                if (ok) {
+                    pv_waited = j;
+                    load_v(j + 1);
+                }
+            }
+            // P V(j): P written by the softmax (and O rescaled), V landed
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(kBarPFull), (uint32_t)(j & 1), abort_flag, lim, 29));
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(kBarV + j % kVStages), (uint32_t)((j / kVStages) & 1),
+                                                         abort_flag, lim, 24));
             if (ok) {
                 v_waited = j + 1;
+                tc_fence_after();
                 issue_pv(base + kOffP, base + kOffV + (uint32_t)(j % kVStages) * kOp, tmem + kColO, idpv, j > 0);
                 mma_commit_warp(bar(kBarPV));
                 pv_issued = j + 1;
             }
         }
-    }
-
-    // ---- epilogue: wait for the last P V, O / l to bf16 ----
-    if (alive) {
-        ok = ok && mbar_wait(bar(kBarPV), (uint32_t)((n - 1) & 1), abort_flag, lim, 25);
-        alive = group_all(kBarGroup, kThreads, ok);
-        if (alive) {
-            pv_waited = n;
+        if (!ok && lane == 0) {
+            // copies and MMAs still in flight land before shared memory and TMEM go away
+            if (q_pending) drain_wait(bar(kBarQ), 0);
+            for (int j = k_waited; j < k_issued; ++j) drain_wait(bar(kBarK + j % kKStages), (uint32_t)((j / kKStages) & 1));
+            for (int j = v_waited; j < v_issued; ++j) drain_wait(bar(kBarV + j % kVStages), (uint32_t)((j / kVStages) & 1));
+            for (int j = s_waited; j < s_issued; ++j) drain_wait(bar(kBarS + (j & 1)), (uint32_t)((j >> 1) & 1));
+            for (int j = pv_waited; j < pv_issued; ++j) drain_wait(bar(kBarPV), (uint32_t)(j & 1));
+        }
+        __syncwarp();
+    } else {
+        // ======================= softmax (warps 0-7) =======================
+        // Threads leave the loop only together, after a vote (bar.red), so the
+        // exchange barrier is never left half-arrived.
+        bool alive = true, ok = true;
+        float m_ref = -INFINITY, l = 0.0f;
+        for (int j = 0; j < n; ++j) {
+            // (the vote on this wait rides on the maximum's exchange barrier below; a thread
+            // whose wait gave up reads scores that are not ready, and the vote then ends the loop)
+            ok = mbar_wait(bar(kBarS + (j & 1)), (uint32_t)((j >> 1) & 1), abort_flag, lim, 22);
             tc_fence_after();
-            xchg[tid] = l;                       // the row sum is the two halves' parts
-            named_bar_sync(kBarGroup, kThreads);
-            const float inv = 1.0f / (xchg[tid] + xchg[tid ^ kBM]);
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) +
-                                  (((size_t)bb * T + (size_t)t) * a.H + h) * (size_t)a.dv;
+            const int s0 = tile_start(j) + kHalfKeys * half;     // this thread's first key
+            const bool sink_tile = j < nA;
+            float x[kHalfKeys];
+#pragma unroll
+            for (int c = 0; c < kHalfKeys / 16; ++c)
+                tmem_ld16(lane_base + kColS + 128u * (j & 1) + (uint32_t)(kHalfKeys * half) + 16u * c,
+                          *reinterpret_cast<float(*)[16]>(&x[16 * c]));
+            // Are all of this thread's keys inside its row's key set?  (Then no per-key mask.)
+            bool full;
+            if (sink_tile) full = s0 + kHalfKeys <= sink;
+            else if (split) full = s0 >= ws && s0 + kHalfKeys <= we;
+            else full = (ws <= sink) ? (s0 + kHalfKeys <= max(sink, we))
+                                     : (s0 + kHalfKeys <= sink || (s0 >= ws && s0 + kHalfKeys <= we));
+            tmem_wait_ld();
+            // this warp is done with the score buffer: the producer may issue tile j + 2 into it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarSFree + (j & 1)));
+            if (!full) {
+#pragma unroll
+                for (int i = 0; i < kHalfKeys; ++i) {
+                    const int s = s0 + i;
+                    const bool valid = sink_tile ? (s < sink)
+                                                 : (s < T && ((!split && s < sink) || (s >= ws && s < we)));
+                    x[i] = valid ? x[i] : -INFINITY;
+                }
+            }
+            // maximum of the raw scores (the scale is positive) over both halves of the row
+            float mx[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) mx[e] = x[e];
+#pragma unroll
+            for (int i = 4; i < kHalfKeys; ++i) mx[i & 3] = fmaxf(mx[i & 3], x[i]);
+            xchg[tid] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            if (!group_all(kBarGroup, kSoftThreads, ok)) { alive = false; break; }
+            const float mt = fmaxf(xchg[tid], xchg[tid ^ kBM]) * a.scale_log2;
+            const bool move = mt > m_ref + kMoveRef;   // the same decision in both threads of the row
+            float alpha = 1.0f;
+            if (move) {
+                alpha = ex2(m_ref - mt);
+                m_ref = mt;
+            }
+            const float neg_mr = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+            float sm[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[kHalfKeys / 2];
+#pragma unroll
+            for (int i = 0; i < kHalfKeys / 2; ++i) {
+                const float p0 = ex2(fmaf(x[2 * i], a.scale_log2, neg_mr));
+                const float p1 = ex2(fmaf(x[2 * i + 1], a.scale_log2, neg_mr));
+                sm[i & 3] += p0 + p1;
+                pk[i] = pack_bf16x2(p0, p1);
+            }
+            const float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);     // this half's part of the row sum
+            l = l * alpha + sum;
+            // ---- the previous P V must be done: P's buffer is reused and O may be rescaled ----
+            if (j > 0) {
+                ok = mbar_wait(bar(kBarPV), (uint32_t)((j - 1) & 1), abort_flag, lim, 23);
+                if (!group_all(kBarGroup, kSoftThreads, ok)) { alive = false; break; }
+                tc_fence_after();
+            }
+            // TMEM loads and stores are warp-collective: the whole warp rescales when any
+            // of its rows moved its reference (the others with alpha = 1)
+            if (__any_sync(0xffffffffu, move && j > 0)) {
+                const float f = (move && j > 0) ? alpha : 1.0f;
 #pragma unroll 1
-            for (int c = c_lo; c < c_hi; ++c) {
-                float o[16];
-                tmem_ld16(lane_base + kColO + 16u * c, o);
-                tmem_wait_ld();
-                if (t < T) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + 16 * c);
-                    dst[0] = make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
-                                        pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
-                    dst[1] = make_uint4(pack_bf16x2(o[8] * inv, o[9] * inv), pack_bf16x2(o[10] * inv, o[11] * inv),
-                                        pack_bf16x2(o[12] * inv, o[13] * inv),
-                                        pack_bf16x2(o[14] * inv, o[15] * inv));
+                for (int c = c_lo; c < c_hi; ++c) {
+                    float o[16];
+                    tmem_ld16(lane_base + kColO + 16u * c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] *= f;
+                    tmem_st16(lane_base + kColO + 16u * c, o);
+                }
+                tmem_wait_st();
+            }
+            // ---- this thread's 64 keys of the P row (bf16) into its box of the K-major SW128 operand ----
+            {
+                const uint32_t prow = base + kOffP + (uint32_t)half * kBox + (uint32_t)row * 128u;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(prow + ((uint32_t)(c ^ (row & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                                 pk[4 * c + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarPFull));
+        }
+
+        // ---- epilogue: wait for the last P V, O / l to bf16 ----
+        if (alive) {
+            ok = mbar_wait(bar(kBarPV), (uint32_t)((n - 1) & 1), abort_flag, lim, 25);
+            alive = group_all(kBarGroup, kSoftThreads, ok);
+            if (alive) {
+                tc_fence_after();
+                xchg[tid] = l;                       // the row sum is the two halves' parts
+                named_bar_sync(kBarGroup, kSoftThreads);
+                const float inv = 1.0f / (xchg[tid] + xchg[tid ^ kBM]);
+                __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) +
+                                      (((size_t)bb * T + (size_t)t) * a.H + h) * (size_t)a.dv;
+#pragma unroll 1
+                for (int c = c_lo; c < c_hi; ++c) {
+                    float o[16];
+                    tmem_ld16(lane_base + kColO + 16u * c, o);
+                    tmem_wait_ld();
+                    if (t < T) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + 16 * c);
+                        dst[0] = make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
+                                            pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
+                        dst[1] = make_uint4(pack_bf16x2(o[8] * inv, o[9] * inv), pack_bf16x2(o[10] * inv, o[11] * inv),
+                                            pack_bf16x2(o[12] * inv, o[13] * inv),
+                                            pack_bf16x2(o[14] * inv, o[15] * inv));
+                    }
                 }
             }
         }
     }
-    if (!alive && warp == 0 && lane == 0) {
-        // copies and MMAs still in flight land before shared memory and TMEM go away
-        if (q_pending) drain_wait(bar(kBarQ), 0);
-        for (int j = k_waited; j < k_issued; ++j) drain_wait(bar(kBarK + j % kKStages), (uint32_t)((j / kKStages) & 1));
-        for (int j = v_waited; j < v_issued; ++j) drain_wait(bar(kBarV + j % kVStages), (uint32_t)((j / kVStages) & 1));
-        for (int j = s_waited; j < s_issued; ++j) drain_wait(bar(kBarS + (j & 1)), (uint32_t)((j >> 1) & 1));
-        for (int j = pv_waited; j < pv_issued; ++j) drain_wait(bar(kBarPV), (uint32_t)(j & 1));
-    }
-    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
