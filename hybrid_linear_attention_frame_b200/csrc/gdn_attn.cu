@@ -44,10 +44,10 @@ constexpr int kKStages = 3, kVStages = 2;
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kOp;
 constexpr uint32_t kOffV = kOffK + kKStages * kOp;
-constexpr uint32_t kOffP = kOffV + kVStages * kOp;
-constexpr uint32_t kOffBar = kOffP + kOp;
-enum : uint32_t { kBarQ = 0, kBarK = 1, kBarV = kBarK + kKStages, kBarS = kBarV + kVStages, kBarPV = kBarS + 2,
-                  kBarSFree = kBarPV + 1,   // [2] the softmax warps have read a score buffer (8 arrivals)
+constexpr uint32_t kOffBar = kOffV + kVStages * kOp;
+enum : uint32_t { kBarQ = 0, kBarK = 1, kBarV = kBarK + kKStages, kBarS = kBarV + kVStages,
+                  kBarPV = kBarS + 2,        // [2] P V of the tile that used P buffer b done
+                  kBarSFree = kBarPV + 2,   // [2] the softmax warps have read a score buffer (8 arrivals)
                   kBarPFull = kBarSFree + 2, // P written and O rescaled (8 arrivals)
                   kNumBars = kBarPFull + 1 };
 __host__ __device__ constexpr uint32_t bar_count(uint32_t i) {
@@ -58,11 +58,12 @@ constexpr uint32_t kOffTmemSlot = kOffAbort + 8u;
 constexpr uint32_t kOffX = kOffTmemSlot + 16u;                 // 256 floats: the two halves' exchange
 constexpr uint32_t kSmemBytes = kOffX + 4u * kSoftThreads + 1024u; // + slack for 1024-byte alignment
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "SW128 tiles need 1024-B alignment");
+static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0, "SW128 tiles need 1024-B alignment");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;                  // two 128-column score buffers
 constexpr uint32_t kColO = 256;                // the d_v-column output accumulator
+constexpr uint32_t kColP = 384;                // two 64-column P buffers: bf16 pairs, the A operand of P V
 constexpr float kMoveRef = 8.0f;               // log2 units: p stays below 2^8
 constexpr uint32_t kBarGroup = 1;              // named barrier of the softmax warps
 
@@ -105,6 +106,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
                  : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32"
+                 " [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                    "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+                    "r"(v[15])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -123,12 +133,24 @@ __device__ __forceinline__ void issue_s(uint32_t q, uint32_t k, uint32_t d, int 
     for (int ks = 0; ks < nks; ++ks) mma_bf16_warp(d, kmaj(kstep(q, ks)), kmaj(kstep(k, ks)), kIdS, ks > 0);
 }
 
-// O[128 x d_v] (+)= P V, K axis = the 128 keys; V read MN-major (rows = keys).
-__device__ __forceinline__ void issue_pv(uint32_t p, uint32_t v, uint32_t d, uint32_t idpv, bool acc) {
+// One tcgen05 MMA whose A operand is in TMEM (row m in lane m, a bf16 pair per column).
+__device__ __forceinline__ void mma_bf16_tmem_a_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                     uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p, e;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
+// O[128 x d_v] (+)= P V, K axis = the 128 keys: P from TMEM (16 keys = 8 columns per
+// step), V read MN-major from shared memory (rows = keys).
+__device__ __forceinline__ void issue_pv(uint32_t p_tmem, uint32_t v, uint32_t d, uint32_t idpv, bool acc) {
 #pragma unroll
     for (int ks = 0; ks < kBN / 16; ++ks)
-        mma_bf16_warp(d, kmaj(kstep(p, ks)), smem_desc(v + (uint32_t)ks * 2048u, kBox, 1024, kSwizzle128), idpv,
-                      (acc || ks > 0) ? 1u : 0u);
+        mma_bf16_tmem_a_warp(d, p_tmem + 8u * (uint32_t)ks, smem_desc(v + (uint32_t)ks * 2048u, kBox, 1024, kSwizzle128),
+                             idpv, (acc || ks > 0) ? 1u : 0u);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -254,7 +276,8 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             // V slot of tile j - 1 takes tile j + 1 once P V(j - 1) is done
             if (ok && j >= 1 && j + 1 < n) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarPV), (uint32_t)((j - 1) & 1), abort_flag, lim, 28));
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarPV + ((j - 1) & 1)), (uint32_t)(((j - 1) >> 1) & 1),
+                                                       abort_flag, lim, 28));
                 if (ok) {
                     pv_waited = j;
                     load_v(j + 1);
@@ -267,8 +290,9 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (ok) {
                 v_waited = j + 1;
                 tc_fence_after();
-                issue_pv(base + kOffP, base + kOffV + (uint32_t)(j % kVStages) * kOp, tmem + kColO, idpv, j > 0);
-                mma_commit_warp(bar(kBarPV));
+                issue_pv(tmem + kColP + 64u * (uint32_t)(j & 1), base + kOffV + (uint32_t)(j % kVStages) * kOp,
+                         tmem + kColO, idpv, j > 0);
+                mma_commit_warp(bar(kBarPV + (j & 1)));
                 pv_issued = j + 1;
             }
         }
@@ -278,7 +302,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int j = k_waited; j < k_issued; ++j) drain_wait(bar(kBarK + j % kKStages), (uint32_t)((j / kKStages) & 1));
             for (int j = v_waited; j < v_issued; ++j) drain_wait(bar(kBarV + j % kVStages), (uint32_t)((j / kVStages) & 1));
             for (int j = s_waited; j < s_issued; ++j) drain_wait(bar(kBarS + (j & 1)), (uint32_t)((j >> 1) & 1));
-            for (int j = pv_waited; j < pv_issued; ++j) drain_wait(bar(kBarPV), (uint32_t)(j & 1));
+            for (int j = pv_waited; j < pv_issued; ++j) drain_wait(bar(kBarPV + (j & 1)), (uint32_t)((j >> 1) & 1));
         }
         __syncwarp();
     } else {
@@ -346,15 +370,18 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             const float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);     // this half's part of the row sum
             l = l * alpha + sum;
-            // ---- the previous P V must be done: P's buffer is reused and O may be rescaled ----
-            if (j > 0) {
-                ok = mbar_wait(bar(kBarPV), (uint32_t)((j - 1) & 1), abort_flag, lim, 23);
-                if (!group_all(kBarGroup, kSoftThreads, ok)) { alive = false; break; }
-                tc_fence_after();
-            }
+            // ---- P buffer j & 1 was used by tile j - 2: its P V must be done; a rescale of O
+            // needs the previous P V (tile j - 1) done as well (P V's complete in order) ----
+            const bool any_move = __any_sync(0xffffffffu, move && j > 0);
+            const int wait_for = any_move ? j - 1 : j - 2;         // (uniform within the warp)
+            ok = (wait_for < 0) ||
+                 mbar_wait(bar(kBarPV + (wait_for & 1)), (uint32_t)((wait_for >> 1) & 1), abort_flag, lim, 23);
+            // (every softmax thread votes here on every tile, whatever it waited for)
+            if (!group_all(kBarGroup, kSoftThreads, ok)) { alive = false; break; }
+            tc_fence_after();
             // TMEM loads and stores are warp-collective: the whole warp rescales when any
             // of its rows moved its reference (the others with alpha = 1)
-            if (__any_sync(0xffffffffu, move && j > 0)) {
+            if (any_move) {
                 const float f = (move && j > 0) ? alpha : 1.0f;
 #pragma unroll 1
                 for (int c = c_lo; c < c_hi; ++c) {
@@ -365,17 +392,15 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int e = 0; e < 16; ++e) o[e] *= f;
                     tmem_st16(lane_base + kColO + 16u * c, o);
                 }
-                tmem_wait_st();
             }
-            // ---- this thread's 64 keys of the P row (bf16) into its box of the K-major SW128 operand ----
+            // ---- this thread's 64 keys of the P row (bf16 pairs) into TMEM: columns
+            // 32 half .. 32 half + 31 of P buffer j & 1 ----
             {
-                const uint32_t prow = base + kOffP + (uint32_t)half * kBox + (uint32_t)row * 128u;
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    st_shared_v4(prow + ((uint32_t)(c ^ (row & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                                 pk[4 * c + 3]);
+                const uint32_t pt = lane_base + kColP + 64u * (uint32_t)(j & 1) + 32u * (uint32_t)half;
+                tmem_st16u(pt, &pk[0]);
+                tmem_st16u(pt + 16u, &pk[16]);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kBarPFull));
@@ -383,7 +408,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
         // ---- epilogue: wait for the last P V, O / l to bf16 ----
         if (alive) {
-            ok = mbar_wait(bar(kBarPV), (uint32_t)((n - 1) & 1), abort_flag, lim, 25);
+            ok = mbar_wait(bar(kBarPV + ((n - 1) & 1)), (uint32_t)(((n - 1) >> 1) & 1), abort_flag, lim, 25);
             alive = group_all(kBarGroup, kSoftThreads, ok);
             if (alive) {
                 tc_fence_after();
