@@ -381,6 +381,38 @@ __device__ __forceinline__ float chunk_decay(const FwdParams& p, int b, int h, i
 // ---------------------------------------------------------------- the kernel
 
 // ---------------------------------------------------------------- UT inverse
+
+// Two floats -> an f16 pair (the first in the low half).  f16 keeps 10 mantissa bits, as
+// tf32 does, and the inverse's entries lie well inside its range.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// D (16x8) += A (16x16, row) * B (16x8, col), f16 inputs, fp32 accumulate.  Lane l
+// holds A rows g, g+8 / columns 2t, 2t+1 (a0, a1) and 2t+8, 2t+9 (a2, a3), B rows 2t, 2t+1
+// (b0) and 2t+8, 2t+9 (b1) of column g, D rows g, g+8 / columns 2t, 2t+1; g = l / 4, t = l % 4.
+__device__ __forceinline__ void mma_f16_16x8x16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One 16-row x 8-column tile of X (16 rows, K columns) * Y (K rows, 8 columns), as element
+// functors, K a multiple of 16: half the tensor-core instructions of the tf32 form.
+template <int K, typename XF, typename YF>
+__device__ __forceinline__ void tile16x8h(float (&d)[4], XF X, YF Y, int lane) {
+    const int g = lane >> 2, t = 2 * (lane & 3);
+#pragma unroll
+    for (int kk = 0; kk < K; kk += 16)
+        mma_f16_16x8x16(d, pack_f16x2(X(g, kk + t), X(g, kk + t + 1)), pack_f16x2(X(g + 8, kk + t), X(g + 8, kk + t + 1)),
+                        pack_f16x2(X(g, kk + t + 8), X(g, kk + t + 9)),
+                        pack_f16x2(X(g + 8, kk + t + 8), X(g + 8, kk + t + 9)),
+                        pack_f16x2(Y(kk + t, g), Y(kk + t + 1, g)), pack_f16x2(Y(kk + t + 8, g), Y(kk + t + 9, g)));
+}
 // (I + A)^{-1} for the 64 x 64 unit lower-triangular I + A (A strictly lower, stored
 // transposed above the diagonal of AXI) into the lower triangle of AXI, by block
 // combination: [[X, 0], [C, Y]]^{-1} = [[X^-1, 0], [-Y^-1 C X^-1, Y^-1]].
@@ -388,8 +420,8 @@ __device__ __forceinline__ float chunk_decay(const FwdParams& p, int b, int h, i
 // Diagonal 16 x 16 blocks and the first level (16 -> 32) on the four A warps (128
 // threads, `st`): forward substitution in fp32, one column per thread, the column of A
 // that a step needs read as four 16-byte vectors (it is a row of the transposed
-// storage); then the two 16 x 16 combinations on mma.sync tf32, one 8-column tile per
-// warp, as in tc::unit_lower_inverse_64.
+// storage); then the two 16 x 16 combinations on mma.sync (f16 in, fp32 accumulate), one
+// 8-column tile per warp.
 __device__ __forceinline__ void inverse_levels01(float* AXI, float* MS, int st) {
     using tc::AAt;
     using tc::XIv;
@@ -421,16 +453,16 @@ __device__ __forceinline__ void inverse_levels01(float* AXI, float* MS, int st) 
     const int pr = pw >> 1, n0 = 8 * (pw & 1);
     const int hi = 16 * (2 * pr + 1), lo = 16 * (2 * pr);
     float m1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    tc::tile16x8<16>(m1, [&](int r, int k) { return AAt(AXI, hi + r, lo + k); },
-                     [&](int k, int n) { return XIv(AXI, lo + k, lo + n0 + n); }, lane);
+    tile16x8h<16>(m1, [&](int r, int k) { return AAt(AXI, hi + r, lo + k); },
+                  [&](int k, int n) { return XIv(AXI, lo + k, lo + n0 + n); }, lane);
     MSw[g * tc::kMS + 2 * t] = m1[0];
     MSw[g * tc::kMS + 2 * t + 1] = m1[1];
     MSw[(g + 8) * tc::kMS + 2 * t] = m1[2];
     MSw[(g + 8) * tc::kMS + 2 * t + 1] = m1[3];
     __syncwarp();
     float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    tc::tile16x8<16>(y, [&](int r, int k) { return XIv(AXI, hi + r, hi + k); },
-                     [&](int k, int n) { return MSw[k * tc::kMS + n]; }, lane);
+    tile16x8h<16>(y, [&](int r, int k) { return XIv(AXI, hi + r, hi + k); },
+                  [&](int k, int n) { return MSw[k * tc::kMS + n]; }, lane);
     AXI[(hi + g) * kXS + lo + n0 + 2 * t] = -y[0];
     AXI[(hi + g) * kXS + lo + n0 + 2 * t + 1] = -y[1];
     AXI[(hi + g + 8) * kXS + lo + n0 + 2 * t] = -y[2];
@@ -446,8 +478,8 @@ __device__ __forceinline__ void inverse_level2(float* AXI, float* C, int w, int 
     using tc::XIv;
     const int g = lane >> 2, t = lane & 3, mt = w >> 2, c0 = 8 * (w & 3);
     float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    tc::tile16x8<32>(c, [&](int r, int k) { return AAt(AXI, 32 + 16 * mt + r, k); },
-                     [&](int k, int n) { return XIv(AXI, k, c0 + n); }, lane);
+    tile16x8h<32>(c, [&](int r, int k) { return AAt(AXI, 32 + 16 * mt + r, k); },
+                  [&](int k, int n) { return XIv(AXI, k, c0 + n); }, lane);
     C[(16 * mt + g) * kCS + c0 + 2 * t] = c[0];
     C[(16 * mt + g) * kCS + c0 + 2 * t + 1] = c[1];
     C[(16 * mt + g + 8) * kCS + c0 + 2 * t] = c[2];
@@ -455,11 +487,11 @@ __device__ __forceinline__ void inverse_level2(float* AXI, float* C, int w, int 
     named_bar_sync(bar_id, kPrepThreads);
     float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     if (mt == 0)
-        tc::tile16x8<16>(y, [&](int r, int k) { return XIv(AXI, 32 + r, 32 + k); },
-                         [&](int k, int n) { return C[k * kCS + c0 + n]; }, lane);
+        tile16x8h<16>(y, [&](int r, int k) { return XIv(AXI, 32 + r, 32 + k); },
+                      [&](int k, int n) { return C[k * kCS + c0 + n]; }, lane);
     else
-        tc::tile16x8<32>(y, [&](int r, int k) { return XIv(AXI, 48 + r, 32 + k); },
-                         [&](int k, int n) { return C[k * kCS + c0 + n]; }, lane);
+        tile16x8h<32>(y, [&](int r, int k) { return XIv(AXI, 48 + r, 32 + k); },
+                      [&](int k, int n) { return C[k * kCS + c0 + n]; }, lane);
     const int r0 = 32 + 16 * mt + g;
     AXI[r0 * kXS + c0 + 2 * t] = -y[0];
     AXI[r0 * kXS + c0 + 2 * t + 1] = -y[1];
