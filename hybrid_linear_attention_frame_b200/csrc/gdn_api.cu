@@ -180,6 +180,97 @@ int run_bidir(const gdn::FwdParams& p, int chunk_len, size_t elem, void* ws, siz
     return to_status(gdn::launch_combine<float>(p, w, L, stream));
 }
 
+// Segment length (tokens) for a host-buffer call cut into about four pieces along T whose
+// copies overlap the computation, or 0 when the call is too small for that to pay.  Pieces
+// start at frame boundaries and at chunk boundaries (multiples of lcm(64, frame_len)).
+int host_segment_len(int T, int frame_len)
+{
+    int64_t a = 64, b = frame_len;
+    while (b) { const int64_t t = a % b; a = b; b = t; }
+    const int64_t unit = 64 / a * (int64_t)frame_len;          // lcm(64, frame_len)
+    if (unit > T / 4 || (int64_t)T < 16384) return 0;
+    const int64_t seg = ((T / 4 + unit - 1) / unit) * unit;
+    return seg < T ? (int)seg : 0;
+}
+
+// Host-buffer forward for B = 1 cut along T into segments: segment i's inputs go up on one
+// stream, its computation (gdn_forward's kernel on that segment, the state carried on the
+// device from the previous segment) runs on the caller's stream, its output comes down on a
+// third, so that the copies of neighbouring segments overlap the computation and each other.
+// The recurrence is the same (the state entering each segment is the exact state after the
+// previous one); only the chunking inside the layer differs from one gdn_forward call.
+int forward_host_pipelined(const gdn::FwdParams& p, int seg, const void* h_q, const void* h_k, const void* h_v,
+                           const float* h_gate_logit, const float* h_beta_logit, const float* h_state_in,
+                           float* h_state_out, void* h_out, int chunk_len, cudaStream_t stream)
+{
+    const int T = p.T, H = p.H, dk = p.dk, dv = p.dv, fl = p.frame_len;
+    const int nseg = (T + seg - 1) / seg;
+    const size_t ns = (size_t)H * dk * dv * sizeof(float);
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[32];
+    int nev = 0;
+    cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+    while (e == cudaSuccess && nev < 2 * nseg + 1 && nev < 32) {
+        e = cudaEventCreateWithFlags(&ev[nev], cudaEventDisableTiming);
+        if (e == cudaSuccess) ++nev;
+    }
+    int st = (e == cudaSuccess && nev == 2 * nseg + 1) ? GDN_OK : GDN_ERR_CUDA;
+    // the caller's earlier work on `stream` comes first (the device buffers may be in use)
+    if (st == GDN_OK && cudaEventRecord(ev[2 * nseg], stream) != cudaSuccess) st = GDN_ERR_CUDA;
+    if (st == GDN_OK && cudaStreamWaitEvent(s_in, ev[2 * nseg], 0) != cudaSuccess) st = GDN_ERR_CUDA;
+    for (int i = 0; st == GDN_OK && i < nseg; ++i) {
+        const int t0 = i * seg, t1 = min(T, t0 + seg), L = t1 - t0;
+        const int f0 = t0 / fl, f1 = (t1 + fl - 1) / fl;
+        const size_t oq = (size_t)t0 * H * dk, ov = (size_t)t0 * H * dv, ob = (size_t)t0 * H;
+        auto up = [&](void* dst, const void* src, size_t bytes) {
+            if (e == cudaSuccess) e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s_in);
+        };
+        e = cudaSuccess;
+        up(static_cast<__nv_bfloat16*>(const_cast<void*>(p.q)) + oq, static_cast<const __nv_bfloat16*>(h_q) + oq,
+           (size_t)L * H * dk * 2);
+        up(static_cast<__nv_bfloat16*>(const_cast<void*>(p.k)) + oq, static_cast<const __nv_bfloat16*>(h_k) + oq,
+           (size_t)L * H * dk * 2);
+        up(static_cast<__nv_bfloat16*>(const_cast<void*>(p.v)) + ov, static_cast<const __nv_bfloat16*>(h_v) + ov,
+           (size_t)L * H * dv * 2);
+        up(const_cast<float*>(p.gate) + (size_t)f0 * H, h_gate_logit + (size_t)f0 * H, (size_t)(f1 - f0) * H * 4);
+        up(const_cast<float*>(p.beta) + ob, h_beta_logit + ob, (size_t)L * H * 4);
+        if (i == 0 && h_state_in) up(p.state_out, h_state_in, ns);
+        if (e == cudaSuccess) e = cudaEventRecord(ev[2 * i], s_in);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, ev[2 * i], 0);
+        if (e != cudaSuccess) { st = GDN_ERR_CUDA; break; }
+        gdn::FwdParams q = p;
+        q.T = L;
+        q.F = f1 - f0;
+        q.q = static_cast<const __nv_bfloat16*>(p.q) + oq;
+        q.k = static_cast<const __nv_bfloat16*>(p.k) + oq;
+        q.v = static_cast<const __nv_bfloat16*>(p.v) + ov;
+        q.gate = p.gate + (size_t)f0 * H;
+        q.beta = p.beta + ob;
+        q.out = static_cast<__nv_bfloat16*>(p.out) + ov;
+        q.state_in = (i == 0) ? (h_state_in ? p.state_out : nullptr) : p.state_out;   // carried in place
+        q.state_out = p.state_out;
+        st = run_bf16(q, chunk_len, stream);
+        if (st != GDN_OK) break;
+        if (cudaEventRecord(ev[2 * i + 1], stream) != cudaSuccess ||
+            cudaStreamWaitEvent(s_out, ev[2 * i + 1], 0) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<__nv_bfloat16*>(h_out) + ov, q.out, (size_t)L * H * dv * 2,
+                            cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
+            st = GDN_ERR_CUDA;
+    }
+    if (st == GDN_OK && h_state_out &&
+        cudaMemcpyAsync(h_state_out, p.state_out, ns, cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
+        st = GDN_ERR_CUDA;
+    // wait for everything enqueued (also after an error), then release the streams and events
+    if (s_out && cudaStreamSynchronize(s_out) != cudaSuccess) st = GDN_ERR_CUDA;
+    if (s_in && cudaStreamSynchronize(s_in) != cudaSuccess) st = GDN_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) st = GDN_ERR_CUDA;
+    for (int j = 0; j < nev; ++j) cudaEventDestroy(ev[j]);
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+    return st;
+}
+
 int forward_host(const void* h_q, const void* h_k, const void* h_v,
                      const float* h_gate_logit, const float* h_beta_logit,
                      const float* h_state_in, float* h_state_out, void* h_out,
@@ -202,6 +293,12 @@ int forward_host(const void* h_q, const void* h_k, const void* h_v,
     const size_t ng = (size_t)B * F * H * sizeof(float);
     const size_t nb = (size_t)B * T * H * sizeof(float);
     const size_t ns = (size_t)B * H * d_k_dim * d_v_dim * sizeof(float);
+    if (!ws && B == 1 && d_state && gdn::seq_supported(d_k_dim, d_v_dim, chunk_len)) {
+        const int seg = host_segment_len(T, frame_len);
+        if (seg > 0)
+            return forward_host_pipelined(p, seg, h_q, h_k, h_v, h_gate_logit, h_beta_logit, h_state_in,
+                                          h_state_out, h_out, chunk_len, stream);
+    }
     cudaError_t e = cudaSuccess;
     if (e == cudaSuccess) e = cudaMemcpyAsync(d_q, h_q, nq, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess) e = cudaMemcpyAsync(d_k, h_k, nq, cudaMemcpyHostToDevice, stream);

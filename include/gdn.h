@@ -158,6 +158,14 @@ int gdn_forward_fp8(const void* q8, const void* k8, const void* v8, float v_scal
  * gdn_forward, copies out (and the final state, if h_state_out is not NULL)
  * back, and waits for the stream.  h_state_in / d_state may be NULL together
  * (zero initial state); d_state is also where the final state is produced.
+ * With B = 1, d_state given, the sequence-parallel kernel's sizes and T of at
+ * least 16,384 tokens and four multiples of lcm(64, frame_len), the call cuts T
+ * into about four segments at such boundaries: each segment's inputs go up on an
+ * internal stream, its computation (the state carried in d_state) runs on
+ * `stream`, its output comes down on another internal stream, so that the copies
+ * overlap the computation and each other.  The result is the same recurrence;
+ * only the chunking differs from one gdn_forward call (rounding-level
+ * differences).  Host buffers should be pinned for the copies to overlap.
  */
 int gdn_forward_host(const void* h_q, const void* h_k, const void* h_v,
                      const float* h_gate_logit, const float* h_beta_logit,

@@ -13,7 +13,7 @@ from workloads import (BLOCK, CLIP241, MINUTE, SESSIONS, TINY, draw, long_memory
                        make_session_blocks)
 
 from gpu_util import (assert_bf16_parity, assert_f32_parity, f32_device, host, run_library,
-                      upload)
+                      upload, rel_l2)
 
 pytestmark = pytest.mark.gpu
 
@@ -181,6 +181,35 @@ def test_host_buffer_entry_matches_device_entry(cuda):
                        Bn, H, T, dk, dk, inp.frame_len, 64)
     np.testing.assert_array_equal(h_out.float().numpy(), o_dev.astype(np.float32))
     np.testing.assert_array_equal(h_state_out.numpy(), s_dev.astype(np.float32))
+
+
+def test_host_buffer_entry_pipelined(cuda):
+    """A clip-length layer (B 1, T 27,280) takes the segmented host path: copies of
+    neighbouring segments overlap the computation, the state carried on the device.
+    Against the oracle at the bf16 bars, and against the device entry (the same
+    recurrence; the warm-up restarts differ, so rounding-level differences only)."""
+    import torch
+    import hybrid_linear_attention_frame_b200 as G
+    w = CLIP241.with_(state_std=0.02)
+    inp = make_inputs(w)
+    o_dev, s_dev = run_library(inp, cuda, state_in=inp.state)
+    q, k, v, g, b = (t.cpu().pin_memory() for t in upload(inp, cuda))
+    Bn, T, H, dk = inp.q.shape
+    h_state = torch.from_numpy(inp.state).pin_memory()
+    h_state_out = torch.empty_like(h_state).pin_memory()
+    h_out = torch.full_like(v, float("nan")).pin_memory()
+    d = [torch.empty_like(x, device=cuda) for x in (q, k, v, g, b)]
+    d_state = torch.empty_like(h_state, device=cuda)
+    d_out = torch.empty_like(v, device=cuda)
+    G.gdn_forward_host(q, k, v, g, b, h_state, h_state_out, h_out, *d, d_state, d_out,
+                       Bn, H, T, dk, dk, inp.frame_len, 64)
+    assert G.gdn_get_last_device_status() == G.GDN_OK
+    o, s = h_out.float().numpy().astype(np.float64), h_state_out.numpy().astype(np.float64)
+    assert not np.isnan(o).any()
+    ro, rs = R.c_forward(inp, inp.state)
+    assert_bf16_parity(o, ro, "pipelined host out")
+    assert_bf16_parity(s, rs, "pipelined host state")
+    assert rel_l2(o, o_dev) <= 1e-3 and rel_l2(s, s_dev) <= 1e-3
 
 
 # ---------------------------------------------------------------- full sizes
