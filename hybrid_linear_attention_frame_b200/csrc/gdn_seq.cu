@@ -992,14 +992,14 @@ gdn_seq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int s = n & 1;
             gram_epilogue(s);
             tc_fence_before();
-            if (qtr < 2) {
-                named_bar_sync(kBarA, 128);      // A complete
-                if (pw == 0 && lane == 0) mbar_arrive(bar(B_GFREE));
-                inverse_levels01(AXI, MSf, 32 * ((pw & 1) | ((pw >> 2) << 1)) + lane);
-            } else {
-                named_bar_sync(kBarP, 128);      // P complete
-                if (pw == 2 && lane == 0) mbar_arrive(bar(B_GFREE));
+            named_bar_sync(kBarPrep, kPrepThreads);      // A and P complete: the Gram is free
+            if (pt == 0) {
+                mbar_arrive(bar(B_GFREE));
+                mbar_arrive(bar(B_GFREE));
             }
+            // the diagonal blocks and the first level on the P warps (their schedulers carry
+            // less of the chain's work than the A warps')
+            if (qtr >= 2) inverse_levels01(AXI, MSf, 32 * ((pw & 1) | ((pw >> 2) << 1)) + lane);
             named_bar_sync(kBarPrep, kPrepThreads);
             inverse_level2(AXI, MSf, pw, lane, kBarPrep);
             bool okw = true;
