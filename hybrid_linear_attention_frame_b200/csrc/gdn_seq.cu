@@ -56,8 +56,6 @@ constexpr int kWarpLoadKQ = 0, kWarpGram = 1, kWarpChainMma = 2, kWarpWU = 3;
 constexpr int kPrepWarp0 = 4, kChainWarp0 = 12;
 constexpr int kPrepThreads = 256;
 constexpr uint32_t kBarPrep = 1;             // named barrier of the prep warps (3: the UT inverse's)
-constexpr uint32_t kBarA = 4;                // the four prep warps that form A and invert I + A
-constexpr uint32_t kBarP = 5;                // the four prep warps that form P
 
 // product of gates over a warm-up stretch below which the state entering it is dropped: 2^-48
 constexpr float kWarmupLogDecay = 48.0f * 0.693147181f;

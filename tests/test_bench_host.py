@@ -88,3 +88,36 @@ def test_softmax_and_bidir_modes_parse():
     assert a.layer == "softmax" and a.direction == "causal"
     a = bench.parse_args(["--direction", "bidir"])
     assert a.layer == "gdn" and a.direction == "bidir"
+
+
+def test_fp8_algorithmic_bytes_are_564_per_token_head():
+    """e4m3 q, k, v: one byte per element in, the bf16 output and the beta logit as before."""
+    w = MINUTE
+    gates = w.B * w.n_frames * w.H * 4
+    assert bench.algorithmic_bytes(w, False, False, in_elem=1) - gates == 564 * w.B * w.T * w.H
+
+
+@pytest.mark.parametrize("argv", [[], ["--inputs", "fp8"], ["--workload", "block"], ["--workload", "sessions"],
+                                  ["--workload", "clip241"], ["--direction", "bidir"], ["--path", "ws"]])
+def test_both_arms_report_the_same_config_keys(argv):
+    """The reference arm and ours build `config` with the same function, so the keys match
+    for every workload and mode (the driver compares them)."""
+    a = bench.parse_args(argv)
+    w = bench.workload_of(a)
+    cfg = bench.run_config(a, w)
+    for key in ("workload", "B", "H", "T", "d_k", "d_v", "frame_len", "chunk_len", "direction",
+                "gate_placement", "api", "inputs"):
+        assert key in cfg, key
+    assert ("gdn_forward_fp8" in cfg["api"]) == ("--inputs" in argv)
+    assert cfg["inputs"].startswith("q, k, v as e4m3") == ("--inputs" in argv)
+
+
+def test_fp8_reference_arm_runs_on_the_widened_inputs():
+    """The reference arm with --inputs fp8 times the oracle on the e4m3 inputs' values and
+    prints the same config as our arm."""
+    a = bench.parse_args(["--impl", "reference", "--inputs", "fp8", "--workload", "block",
+                          "--steps", "1", "--warmup", "0", "--cpu-seconds", "0.2"])
+    w = bench.workload_of(a)
+    line = bench.run_reference(a, w, 0, 1)
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["config"] == bench.run_config(a, w)
