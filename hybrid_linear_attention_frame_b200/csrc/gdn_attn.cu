@@ -9,19 +9,20 @@
 //
 // the sink frames, the cached blocks and the whole current block.
 //
-// One CTA of 256 threads per (128 queries, head, batch entry); threads r and r + 128
-// share query row r (TMEM lane r), each taking 64 of a tile's keys and half of the
-// output columns.  For each key tile of 128 tokens:
+// One CTA of 544 threads per (128 queries, head, batch entry); threads r, r + 128,
+// r + 256 and r + 384 share query row r (TMEM lane r), each taking 32 of a tile's keys
+// and a quarter of the output columns.  For each key tile of 128 tokens:
 //   S = Q K^T on the tensor cores into TMEM (two buffers: the next tile's S runs
 //     while this tile's softmax does),
 //   the softmax in registers against a lazily moved reference maximum (it moves
 //     only when a score exceeds it by more than 2^8, so the accumulator is rarely
 //     rescaled; the final division by the running sum makes the result exact
-//     whatever reference was used),
-//   P in bf16 to shared memory, O += P V on the tensor cores into TMEM.
+//     whatever reference was used), the row's maximum exchanged once per tile,
+//   P in bf16 pairs into TMEM (two buffers), O += P V on the tensor cores into TMEM
+//     with P as the A operand.
 // K tiles are triple-buffered and V tiles double-buffered, loaded by TMA (128-byte
 // swizzle, rows past the end of the sequence read as zeros and are masked).
-// Warp 8 issues the copies and the MMAs; warps 0-7 only run the softmax, and the two
+// Warp 16 issues the copies and the MMAs; warps 0-15 only run the softmax, and the two
 // sides meet at mbarriers: S ready / S read, P written / P V done.  Every wait is
 // bounded.
 #include "gdn_common.cuh"
@@ -32,12 +33,15 @@ namespace attn {
 
 using namespace sm100;
 
-constexpr int kSoftThreads = 256;              // softmax warps 0-7: two threads per query row
-constexpr int kProducerWarp = 8;               // copies and MMAs
-constexpr int kThreads = kSoftThreads + 32;
-constexpr int kHalfKeys = 64;                  // keys of a tile per thread
 constexpr int kBM = 128;                       // queries per CTA
 constexpr int kBN = 128;                       // keys per tile
+constexpr int kParts = 4;                      // softmax threads per query row (four softmax warps
+                                               // per sub-partition hide more of its latency than two)
+constexpr int kSoftThreads = kParts * kBM;     // softmax warps 0 .. 4 kParts - 1
+constexpr int kProducerWarp = kSoftThreads / 32;   // copies and MMAs
+constexpr int kThreads = kSoftThreads + 32;
+constexpr int kKeysPer = kBN / kParts;         // keys of a tile per softmax thread
+static_assert(kKeysPer % 32 == 0, "whole 16-column P stores");
 constexpr uint32_t kBox = 128u * 128u;         // one 64-column SW128 box of 128 rows: 16 KB
 constexpr uint32_t kOp = 2u * kBox;            // a 128 x (d <= 128) operand: two boxes
 constexpr int kKStages = 3, kVStages = 2;
@@ -51,11 +55,11 @@ enum : uint32_t { kBarQ = 0, kBarK = 1, kBarV = kBarK + kKStages, kBarS = kBarV 
                   kBarPFull = kBarSFree + 2, // P written and O rescaled (8 arrivals)
                   kNumBars = kBarPFull + 1 };
 __host__ __device__ constexpr uint32_t bar_count(uint32_t i) {
-    return (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull) ? 8u : 1u;
+    return (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull) ? (uint32_t)(kSoftThreads / 32) : 1u;
 }
 constexpr uint32_t kOffAbort = kOffBar + 8u * kNumBars;
 constexpr uint32_t kOffTmemSlot = kOffAbort + 8u;
-constexpr uint32_t kOffX = kOffTmemSlot + 16u;                 // 256 floats: the two halves' exchange
+constexpr uint32_t kOffX = kOffTmemSlot + 16u;                 // one float per softmax thread: the row parts' exchange
 constexpr uint32_t kSmemBytes = kOffX + 4u * kSoftThreads + 1024u; // + slack for 1024-byte alignment
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0, "SW128 tiles need 1024-B alignment");
@@ -92,6 +96,33 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+
+// A three-input maximum, and pairs of f32 packed in 64-bit registers for the paired FMA and
+// add (one instruction does the work of two): they trim the softmax's instruction count.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t r, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
@@ -180,8 +211,8 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int n = nA + (w_hi - startB + kBN - 1) / kBN;
     auto tile_start = [&](int j) { return j < nA ? kBN * j : startB + kBN * (j - nA); };
 
-    // ---- this thread's query row, half of the keys and its row's key set ----
-    const int row = tid & (kBM - 1), half = (tid / kBM) & 1;      // (softmax threads)
+    // ---- this thread's query row, its part of the keys and its row's key set ----
+    const int row = tid & (kBM - 1), part = (tid / kBM) % kParts;   // (softmax threads)
     const int t = t0 + row;
     const int te = min(t, T - 1);
     const int ws = max(0, te / bl - a.cached) * bl;
@@ -205,7 +236,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gb + kOffTmemSlot);
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);   // warp w reads lanes 32 (w % 4) ..
     float* xchg = reinterpret_cast<float*>(gb + kOffX);
-    const int nco = a.dv / 16, c_lo = half ? (nco + 1) / 2 : 0, c_hi = half ? nco : (nco + 1) / 2;
+    const int nco = a.dv / 16, c_lo = part * nco / kParts, c_hi = (part + 1) * nco / kParts;
     const uint32_t idpv = idesc_bf16(128, a.dv, false, true);
     const int nks = a.dk / 16;
 
@@ -316,19 +347,19 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // whose wait gave up reads scores that are not ready, and the vote then ends the loop)
             ok = mbar_wait(bar(kBarS + (j & 1)), (uint32_t)((j >> 1) & 1), abort_flag, lim, 22);
             tc_fence_after();
-            const int s0 = tile_start(j) + kHalfKeys * half;     // this thread's first key
+            const int s0 = tile_start(j) + kKeysPer * part;      // this thread's first key
             const bool sink_tile = j < nA;
-            float x[kHalfKeys];
+            float x[kKeysPer];
 #pragma unroll
-            for (int c = 0; c < kHalfKeys / 16; ++c)
-                tmem_ld16(lane_base + kColS + 128u * (j & 1) + (uint32_t)(kHalfKeys * half) + 16u * c,
+            for (int c = 0; c < kKeysPer / 16; ++c)
+                tmem_ld16(lane_base + kColS + 128u * (j & 1) + (uint32_t)(kKeysPer * part) + 16u * c,
                           *reinterpret_cast<float(*)[16]>(&x[16 * c]));
             // Are all of this thread's keys inside its row's key set?  (Then no per-key mask.)
             bool full;
-            if (sink_tile) full = s0 + kHalfKeys <= sink;
-            else if (split) full = s0 >= ws && s0 + kHalfKeys <= we;
-            else full = (ws <= sink) ? (s0 + kHalfKeys <= max(sink, we))
-                                     : (s0 + kHalfKeys <= sink || (s0 >= ws && s0 + kHalfKeys <= we));
+            if (sink_tile) full = s0 + kKeysPer <= sink;
+            else if (split) full = s0 >= ws && s0 + kKeysPer <= we;
+            else full = (ws <= sink) ? (s0 + kKeysPer <= max(sink, we))
+                                     : (s0 + kKeysPer <= sink || (s0 >= ws && s0 + kKeysPer <= we));
             tmem_wait_ld();
             // this warp is done with the score buffer: the producer may issue tile j + 2 into it
             tc_fence_before();
@@ -336,7 +367,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (lane == 0) mbar_arrive(bar(kBarSFree + (j & 1)));
             if (!full) {
 #pragma unroll
-                for (int i = 0; i < kHalfKeys; ++i) {
+                for (int i = 0; i < kKeysPer; ++i) {
                     const int s = s0 + i;
                     const bool valid = sink_tile ? (s < sink)
                                                  : (s < T && ((!split && s < sink) || (s >= ws && s < we)));
@@ -344,14 +375,15 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             }
             // maximum of the raw scores (the scale is positive) over both halves of the row
-            float mx[4];
+            float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) mx[e] = x[e];
-#pragma unroll
-            for (int i = 4; i < kHalfKeys; ++i) mx[i & 3] = fmaxf(mx[i & 3], x[i]);
+            for (int q = 0; q < (kKeysPer - 4) / 2; ++q) mx[q & 3] = max3f(mx[q & 3], x[4 + 2 * q], x[5 + 2 * q]);
             xchg[tid] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             if (!group_all(kBarGroup, kSoftThreads, ok)) { alive = false; break; }
-            const float mt = fmaxf(xchg[tid], xchg[tid ^ kBM]) * a.scale_log2;
+            float mrow = xchg[row];
+#pragma unroll
+            for (int q = 1; q < kParts; ++q) mrow = fmaxf(mrow, xchg[row + kBM * q]);
+            const float mt = mrow * a.scale_log2;
             const bool move = mt > m_ref + kMoveRef;   // the same decision in both threads of the row
             float alpha = 1.0f;
             if (move) {
@@ -359,16 +391,21 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 m_ref = mt;
             }
             const float neg_mr = (m_ref == -INFINITY) ? 0.0f : -m_ref;
-            float sm[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[kHalfKeys / 2];
+            const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(neg_mr, neg_mr);
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};        // (+0, +0) pairs
+            uint32_t pk[kKeysPer / 2];
 #pragma unroll
-            for (int i = 0; i < kHalfKeys / 2; ++i) {
-                const float p0 = ex2(fmaf(x[2 * i], a.scale_log2, neg_mr));
-                const float p1 = ex2(fmaf(x[2 * i + 1], a.scale_log2, neg_mr));
-                sm[i & 3] += p0 + p1;
+            for (int i = 0; i < kKeysPer / 2; ++i) {
+                float t0, t1;
+                f2unpack(fma2(f2pack(x[2 * i], x[2 * i + 1]), sc2, nm2), t0, t1);
+                const float p0 = ex2(t0), p1 = ex2(t1);
+                acc[i & 3] = add2(acc[i & 3], f2pack(p0, p1));
                 pk[i] = pack_bf16x2(p0, p1);
             }
-            const float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);     // this half's part of the row sum
+            float sm[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) f2unpack(acc[e], sm[2 * e], sm[2 * e + 1]);
+            const float sum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
             l = l * alpha + sum;
             // ---- P buffer j & 1 was used by tile j - 2: its P V must be done; a rescale of O
             // needs the previous P V (tile j - 1) done as well (P V's complete in order) ----
@@ -393,12 +430,12 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     tmem_st16(lane_base + kColO + 16u * c, o);
                 }
             }
-            // ---- this thread's 64 keys of the P row (bf16 pairs) into TMEM: columns
-            // 32 half .. 32 half + 31 of P buffer j & 1 ----
+            // ---- this thread's keys of the P row (bf16 pairs) into TMEM: columns
+            // kKeysPer/2 part .. of P buffer j & 1 ----
             {
-                const uint32_t pt = lane_base + kColP + 64u * (uint32_t)(j & 1) + 32u * (uint32_t)half;
-                tmem_st16u(pt, &pk[0]);
-                tmem_st16u(pt + 16u, &pk[16]);
+                const uint32_t pt = lane_base + kColP + 64u * (uint32_t)(j & 1) + (uint32_t)(kKeysPer / 2 * part);
+#pragma unroll
+                for (int c = 0; c < kKeysPer / 32; ++c) tmem_st16u(pt + 16u * c, &pk[16 * c]);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -412,9 +449,12 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             alive = group_all(kBarGroup, kSoftThreads, ok);
             if (alive) {
                 tc_fence_after();
-                xchg[tid] = l;                       // the row sum is the two halves' parts
+                xchg[tid] = l;                       // the row sum is the sum of its parts
                 named_bar_sync(kBarGroup, kSoftThreads);
-                const float inv = 1.0f / (xchg[tid] + xchg[tid ^ kBM]);
+                float lrow = 0.0f;
+#pragma unroll
+                for (int q = 0; q < kParts; ++q) lrow += xchg[row + kBM * q];
+                const float inv = 1.0f / lrow;
                 __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) +
                                       (((size_t)bb * T + (size_t)t) * a.H + h) * (size_t)a.dv;
 #pragma unroll 1

@@ -56,6 +56,8 @@ CASES = {
     "single token": (1, 4, 1, 112, 112, 880, 3, 2, 1),
     "sub-tile sequence": (2, 2, 57, 112, 112, 10, 3, 2, 1),
     "sink inside the window, long blocks": (1, 2, 1300, 112, 112, 200, 3, 2, 1),
+    "two whole query tiles": (1, 2, 256, 112, 112, 40, 2, 1, 1),
+    "one row in the second query tile": (1, 2, 129, 112, 112, 20, 3, 2, 1),
 }
 
 

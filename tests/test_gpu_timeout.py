@@ -8,8 +8,9 @@ producer is simply slower than the bound).  Under a bound below 1 ms the mbarrie
 waits poll without a suspend hint and read the clock on every poll, and the ring
 kernel's counter waits read it every ~1 us, so every kernel reports the timeout:
 the ring kernel (gdn_forward_ws), the sequence-parallel kernel (gdn_forward at
-d 112, and its e4m3-input instance through gdn_forward_fp8) and the fused chunk
-kernel (gdn_forward at d 128).  Each kernel then
+d 112, and its e4m3-input instance through gdn_forward_fp8), the fused chunk
+kernel (gdn_forward at d 128) and the softmax-attention kernel
+(gdn_softmax_attention).  Each kernel then
 drains the copies and MMAs it has in flight and returns.  After each such call
 the default bound is restored and a normal call must match the untouched
 reference outputs bit for bit.
@@ -49,13 +50,18 @@ def _run(G, entry, tensors, inp, ws):
         G.gdn_forward_ws(q, k, v, g, b, s_in, s, o, Bn, H, T, dk, dv, inp.frame_len, 64, ws)
     elif entry == "fp8":
         G.gdn_forward_fp8(q, k, v, inp.v_scale, g, b, s_in, s, o, Bn, H, T, dk, dv, inp.frame_len, 64)
+    elif entry == "attn":
+        # the softmax-attention kernel (no state: s stays as filled)
+        s.zero_()
+        G.gdn_softmax_attention(q, k, v, o, Bn, H, T, dk, dv, inp.frame_len, 3, 2, 1)
     else:
         G.gdn_forward(q, k, v, g, b, s_in, s, o, Bn, H, T, dk, dv, inp.frame_len, 64)
     return o, s, G.gdn_get_last_device_status()
 
 
-@pytest.mark.parametrize("entry,d,path", [("ws", 112, None), ("plain", 112, 2), ("plain", 128, 1), ("fp8", 112, 2)],
-                         ids=["ring", "sequence_parallel", "fused_d128", "sequence_parallel_e4m3"])
+@pytest.mark.parametrize("entry,d,path", [("ws", 112, None), ("plain", 112, 2), ("plain", 128, 1), ("fp8", 112, 2),
+                                          ("attn", 112, None)],
+                         ids=["ring", "sequence_parallel", "fused_d128", "sequence_parallel_e4m3", "softmax_attention"])
 def test_wait_timeout_is_reported_and_context_recovers(cuda, entry, d, path):
     import torch
     import hybrid_linear_attention_frame_b200 as G
