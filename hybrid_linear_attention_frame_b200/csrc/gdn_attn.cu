@@ -51,11 +51,14 @@ constexpr uint32_t kOffV = kOffK + kKStages * kOp;
 constexpr uint32_t kOffBar = kOffV + kVStages * kOp;
 enum : uint32_t { kBarQ = 0, kBarK = 1, kBarV = kBarK + kKStages, kBarS = kBarV + kVStages,
                   kBarPV = kBarS + 2,        // [2] P V of the tile that used P buffer b done
-                  kBarSFree = kBarPV + 2,   // [2] the softmax warps have read a score buffer (8 arrivals)
-                  kBarPFull = kBarSFree + 2, // P written and O rescaled (8 arrivals)
-                  kNumBars = kBarPFull + 1 };
+                  kBarSFree = kBarPV + 2,   // [2] the softmax warps have read a score buffer (one arrival each)
+                  // [2] P buffer b written and O rescaled (one arrival per softmax warp).  Per
+                  // buffer: the softmax can finish tile j + 1 before the issuing warp looks for
+                  // tile j, but not tile j + 2 (its P waits for P V(j), issued after that look)
+                  kBarPFull = kBarSFree + 2,
+                  kNumBars = kBarPFull + 2 };
 __host__ __device__ constexpr uint32_t bar_count(uint32_t i) {
-    return (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull) ? (uint32_t)(kSoftThreads / 32) : 1u;
+    return (i >= kBarSFree && i < kBarPFull + 2) ? (uint32_t)(kSoftThreads / 32) : 1u;
 }
 constexpr uint32_t kOffAbort = kOffBar + 8u * kNumBars;
 constexpr uint32_t kOffTmemSlot = kOffAbort + 8u;
@@ -315,7 +318,8 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             }
             // P V(j): P written by the softmax (and O rescaled), V landed
-            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(kBarPFull), (uint32_t)(j & 1), abort_flag, lim, 29));
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(kBarPFull + (j & 1)), (uint32_t)((j >> 1) & 1), abort_flag,
+                                                         lim, 29));
             ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(kBarV + j % kVStages), (uint32_t)((j / kVStages) & 1),
                                                          abort_flag, lim, 24));
             if (ok) {
@@ -440,7 +444,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarPFull));
+            if (lane == 0) mbar_arrive(bar(kBarPFull + (j & 1)));
         }
 
         // ---- epilogue: wait for the last P V, O / l to bf16 ----
