@@ -90,9 +90,13 @@ class _World:
 _SEQ_COUNTS = dict(SREADY=8, PEGO=8, EREADY=4, OREADY=4, WREADY=4, FULL0=2, FULL1=2, GFREE=2)
 
 
-def _seq_run(N, seed, mutation=None):
+def _seq_run(N, seed, mutation=None, early_release=False):
     """One stretch of N chunks (bf16 path): loader, Gram, W/U, chain-MMA, prep (as one
-    role: its eight warps meet at named barriers) and the eight chain/output warps."""
+    role: its eight warps meet at named barriers) and the eight chain/output warps.
+    The kernel releases a stage (K, Q, -W, scalars and its P tile) once P E has run.
+    early_release models the alternative measured slower on the GPU: the stage
+    released once MMA2 has read it, the P tile separately after P E (PFREE), and
+    e^G/|q| read by the output warps as soon as READY arrives."""
     w = _World(lambda name: _SEQ_COUNTS.get(name, 1), random.Random(seed))
     ready = (lambda s: "READY") if mutation == "one READY barrier" else (lambda s: f"READY{s}")
     ready_ph = (lambda n: n) if mutation == "one READY barrier" else (lambda n: n >> 1)
@@ -106,8 +110,8 @@ def _seq_run(N, seed, mutation=None):
             if n >= 2:
                 if mutation != "no SFREE wait":
                     yield from w.wait(f"SFREE{s}", (n - 2) >> 1)
-                # the stage's K, Q, W and scalars are rewritten
-                w.need(("gram", n - 2), ("wu", n - 2), ("m1", n - 2), ("m2", n - 2), ("pe", n - 2))
+                # the stage's K, Q, W and gate scalars are rewritten
+                w.need(("gram", n - 2), ("wu", n - 2), ("m1", n - 2), ("m2", n - 2))
             w.async_op("loader", ("kq", n), [f"FULL{s}"])    # expect_tx arrival + the copy
             yield
             w.arrive(f"FULL{s}")                             # the gate scan written
@@ -149,15 +153,22 @@ def _seq_run(N, seed, mutation=None):
             yield from w.wait("EREADY", n)
             if n > 0:
                 w.need(*(("rb", n - 1, q) for q in range(8)))   # SACC read back and decayed
-            w.async_op("cm", ("m2", n), ["M2"])
+            w.async_op("cm", ("m2", n), ["M2"] + ([f"SFREE{s}"] if early_release else []))
             yield from w.wait("PEGO", n)
-            w.async_op("cm", ("pe", n), ["PEDONE", f"SFREE{s}"])
+            w.async_op("cm", ("pe", n), ["PEDONE"] + ([f"PFREE{s}"] if early_release else [f"SFREE{s}"]))
 
     def prep():
         for n in range(N):
             s = n & 1
             yield from w.wait(f"FULL{s}", n >> 1)
             yield from w.wait("G1", n)
+            yield
+            if n >= 2:
+                # the chunk's per-row scalars (1/|k| e^{G_L-G}, e^G/|q|) into the stage
+                w.need(*(("dl", n - 2, q) for q in range(4, 8)), *(("gq", n - 2, q) for q in range(4)))
+            w.done.add(("cs", n))
+            if n >= 2 and early_release and mutation != "no PFREE wait":
+                yield from w.wait(f"PFREE{s}", (n - 2) >> 1)
             yield
             if n >= 2:
                 w.need(("pe", n - 2))                # P[s] rewritten
@@ -178,6 +189,9 @@ def _seq_run(N, seed, mutation=None):
             s = n & 1
             last = n == N - 1
             yield from w.wait(ready(s), ready_ph(n))
+            if A and early_release and mutation != "late GQ read":
+                w.need(("cs", n))
+                w.done.add(("gq", n, q))             # e^G/|q| of the rows read at once
             if A:
                 yield from w.wait(f"WU{s}", n >> 1)
                 yield
@@ -186,6 +200,8 @@ def _seq_run(N, seed, mutation=None):
             if not A:
                 if n > 0:
                     w.need(("m2", n - 1))            # E' tile rewritten
+                w.need(("cs", n))
+                w.done.add(("dl", n, q))             # 1/|k| e^{G_L-G} read for E'
                 yield
                 w.arrive("EREADY")
                 if n > 0:
@@ -194,6 +210,9 @@ def _seq_run(N, seed, mutation=None):
                 yield
             else:
                 yield
+                if not (early_release and mutation != "late GQ read"):
+                    w.need(("cs", n))
+                    w.done.add(("gq", n, q))         # e^G/|q| read for the Q S scaling
             w.arrive("PEGO")
             if not last:
                 yield from w.wait(f"FULL{(n + 1) & 1}", (n + 1) >> 1)
@@ -219,18 +238,20 @@ def _seq_run(N, seed, mutation=None):
 
 
 @pytest.mark.parametrize("N", [1, 2, 3, 5, 8])
-def test_seq_kernel_protocol(N):
+@pytest.mark.parametrize("early_release", [False, True], ids=["stage_after_pe", "stage_after_mma2"])
+def test_seq_kernel_protocol(N, early_release):
     for seed in range(60):
-        _seq_run(N, seed)
+        _seq_run(N, seed, early_release=early_release)
 
 
 @pytest.mark.parametrize("mutation", ["no SFREE wait", "one READY barrier", "no GFREE wait", "no VFREE wait",
-                                      "no TREADY wait"])
+                                      "no TREADY wait", "no PFREE wait", "late GQ read"])
 def test_seq_kernel_protocol_model_catches_planted_mistakes(mutation):
+    early = mutation in ("no PFREE wait", "late GQ read")     # mistakes of the early-release form
     caught = 0
     for seed in range(60):
         try:
-            _seq_run(5, seed, mutation)
+            _seq_run(5, seed, mutation, early_release=early)
         except AssertionError:
             caught += 1
     assert caught > 0, f"the model missed: {mutation}"
