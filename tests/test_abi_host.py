@@ -224,3 +224,28 @@ def test_softmax_attention_validates_before_any_device_work():
                                      None) == G.GDN_ERR_INVALID_ARG
     # T = 0: nothing to do, nothing enqueued
     assert lib.gdn_softmax_attention(*args, 1, 2, 0, 112, 112, 16, 3, 2, 1, None) == G.GDN_OK
+
+
+def test_fp8_entry_validates_before_any_device_work():
+    """gdn_forward_fp8 rejects a bad scale, unsupported sizes, null, misaligned or
+    overlapping buffers on the host (fake device addresses, never dereferenced)."""
+    lib = G.load()
+
+    def call(q8=A, k8=2 * A, v8=3 * A, v_scale=0.5, out=6 * A, state_in=None, state_out=None,
+             B=1, H=2, T=64, d=32, frame_len=16, chunk_len=64):
+        return lib.gdn_forward_fp8(q8, k8, v8, v_scale, 4 * A, 5 * A, state_in, state_out, out,
+                                   B, H, T, d, d, frame_len, chunk_len, None)
+
+    for bad in (-1.0, float("nan"), float("inf"), -1e-30):
+        assert call(v_scale=bad) == G.GDN_ERR_INVALID_ARG, bad
+    assert call(d=128) == G.GDN_ERR_UNSUPPORTED            # above the e4m3 kernel's 112
+    assert call(chunk_len=32) == G.GDN_ERR_UNSUPPORTED
+    assert call(q8=None) == G.GDN_ERR_INVALID_ARG
+    assert call(v8=None) == G.GDN_ERR_INVALID_ARG
+    assert call(out=None) == G.GDN_ERR_INVALID_ARG
+    assert call(k8=2 * A + 8) == G.GDN_ERR_INVALID_ARG    # not 16-byte aligned
+    # out is bf16: 2 bytes per element against the inputs' 1, so it reaches v8 from below
+    n = 1 * 64 * 2 * 32
+    assert call(out=3 * A - n) == G.GDN_ERR_INVALID_ARG
+    assert call(B=0) == G.GDN_ERR_INVALID_ARG
+    assert call(frame_len=0) == G.GDN_ERR_INVALID_ARG
