@@ -90,13 +90,20 @@ class _World:
 _SEQ_COUNTS = dict(SREADY=8, PEGO=8, EREADY=4, OREADY=4, WREADY=4, FULL0=2, FULL1=2, GFREE=2)
 
 
-def _seq_run(N, seed, mutation=None, early_release=False):
+def _seq_run(N, seed, mutation=None, early_release=False, pieces=None):
     """One stretch of N chunks (bf16 path): loader, Gram, W/U, chain-MMA, prep (as one
     role: its eight warps meet at named barriers) and the eight chain/output warps.
     The kernel releases a stage (K, Q, -W, scalars and its P tile) once P E has run.
     early_release models the alternative measured slower on the GPU: the stage
     released once MMA2 has read it, the P tile separately after P E (PFREE), and
-    e^G/|q| read by the output warps as soon as READY arrives."""
+    e^G/|q| read by the output warps as soon as READY arrives.
+    pieces: lengths of the chains' pieces the CTA runs one after another (default one
+    piece of N chunks); a piece's last chunk writes the state out instead of handing
+    it on, and the next piece starts from its own initial state (chain_init)."""
+    pieces = pieces or [N]
+    assert sum(pieces) == N
+    starts = {sum(pieces[:i]) for i in range(len(pieces))}
+    ends = {sum(pieces[:i + 1]) - 1 for i in range(len(pieces))}
     w = _World(lambda name: _SEQ_COUNTS.get(name, 1), random.Random(seed))
     ready = (lambda s: "READY") if mutation == "one READY barrier" else (lambda s: f"READY{s}")
     ready_ph = (lambda n: n) if mutation == "one READY barrier" else (lambda n: n >> 1)
@@ -187,7 +194,14 @@ def _seq_run(N, seed, mutation=None, early_release=False):
         A = q < 4                                    # TMEM lanes 0-63; q == 0 stores the output
         for n in range(N):
             s = n & 1
-            last = n == N - 1
+            last = n in ends
+            if n in starts and n > 0:
+                # chain_init: the S tile and SACC from the new piece's initial state
+                w.need(("m1", n - 1), ("m2", n - 1))
+                yield
+                w.done.add(("rb", n - 1, q))
+                w.done.add(("sread", n))
+                w.arrive("SREADY")
             yield from w.wait(ready(s), ready_ph(n))
             if A and early_release and mutation != "late GQ read":
                 w.need(("cs", n))
@@ -242,6 +256,13 @@ def _seq_run(N, seed, mutation=None, early_release=False):
 def test_seq_kernel_protocol(N, early_release):
     for seed in range(60):
         _seq_run(N, seed, early_release=early_release)
+
+
+@pytest.mark.parametrize("pieces", [[1, 1], [2, 3], [1, 4, 1], [3, 1, 2, 2]])
+def test_seq_kernel_protocol_across_pieces(pieces):
+    """A CTA's stretch spans the tail of one chain, whole chains and the head of another."""
+    for seed in range(60):
+        _seq_run(sum(pieces), seed, pieces=pieces)
 
 
 @pytest.mark.parametrize("mutation", ["no SFREE wait", "one READY barrier", "no GFREE wait", "no VFREE wait",
